@@ -1,0 +1,439 @@
+#!/usr/bin/env python3
+"""Benchmark of the fine-grained-scaled FP8 GEMM on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one GEMM call over the headline workload (the decode-shaped dense
+problem M=128, N=2112, K=7168, the shape the DeepGEMM pages quote their
+largest speed-up on) with inputs resident in HBM.  L2 is flushed (a 512 MiB
+write) before every timed launch and each launch is timed alone with CUDA
+events on its stream.  Rank 0 prints one JSON line with the headline value,
+a roofline object for the GEMM kernel, the end-to-end number through the
+public API with host buffers, the CPU oracle as a baseline, the SM clocks seen
+under load and the per-shape numbers of all five workloads.
+
+With N>1 (torchrun, one process per GPU) each rank runs its own replica of
+the workload (the dense GEMM has no exchange step: replicas only), the time is
+the max over ranks and the value counts the work of all ranks.
+
+--impl reference times the CPU oracle (the only reference that exists for
+this method) on the same workload and metric, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dg_inputs as gi  # noqa: E402
+
+METRIC = "FP8 TFLOPS per shape and % of 1-GPU roofline (dense, contiguous, masked MoE)"
+HEADLINE = "dense_decode"
+L2_FLUSH_BYTES = 512 << 20
+
+
+# ------------------------------------------------------------------ helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            mp = json.load(f)
+        return dict(hbm_gbs=float(mp["hbm_gbs"]), bf16_tflops=float(mp["bf16_tflops"]),
+                    bf16_sustained=float(mp.get("bf16_tflops_sustained", mp["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def workload_cost(p):
+    """Algorithmic FLOPs and bytes (each tensor moved once; valid rows only)."""
+    kind = p["kind"]
+    K, N = p["K"], p["N"]
+    nkb = K // 128
+    nbn = (N + 127) // 128
+    if kind == "dense":
+        M = p["M"]
+        flop = 2.0 * M * N * K
+        byts = M * K + N * K + 4 * M * nkb + 4 * nbn * nkb + 2 * M * N
+        rows = M
+    elif kind == "contiguous":
+        rows = int((p["m_indices"] >= 0).sum())
+        G = p["G"]
+        flop = 2.0 * rows * N * K
+        byts = rows * K + G * N * K + 4 * rows * nkb + 4 * G * nbn * nkb + 2 * rows * N + 4 * p["M"]
+    else:
+        G = p["G"]
+        rows = int(np.minimum(p["masked_m"], p["max_m"]).sum())
+        flop = 2.0 * rows * N * K
+        byts = rows * K + G * N * K + 4 * rows * nkb + 4 * G * nbn * nkb + 2 * rows * N + 4 * G
+    return flop, float(byts), rows
+
+
+def roofline(flop, byts, pk):
+    fp8_peak = 2.0 * pk["bf16_tflops"]  # nominal fp8/bf16 dense ratio 4.5/2.25
+    t_tensor = flop / (fp8_peak * 1e12)
+    t_hbm = byts / (pk["hbm_gbs"] * 1e9)
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    return bound, max(t_tensor, t_hbm), fp8_peak
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "moe_grouped_gemm_wt_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t.get(workload)
+        if e and e.get("kernel_hash") == kernel_hash():
+            return float(e["dram_bytes_per_launch"])
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling while the GPU is busy."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.dev), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        samples = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                samples.append(dict(sm=float(parts[0]), smmax=float(parts[1]),
+                                    power=float(parts[2]), util=float(parts[3]),
+                                    hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        if not samples:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=[], samples=0)
+        busy = [s for s in samples if s["util"] >= 30] or samples
+        reasons = set()
+        for s in busy:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if s[key].lower() == "active":
+                    reasons.add(name)
+        return dict(sm_mhz=statistics.median(s["sm"] for s in busy),
+                    sm_max_mhz=max(s["smmax"] for s in busy),
+                    reasons=sorted(reasons), samples=len(busy))
+
+
+# ------------------------------------------------------------ our library
+
+def to_device(p, torch, dev):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    out = dict(A=t(p["A"]), B=t(p["B"]), sA=t(gi.sa_to_kernel_layout(p["sA"])), sB=t(p["sB"]))
+    if p["kind"] == "dense":
+        out["D"] = torch.empty((p["M"], p["N"]), dtype=torch.bfloat16, device=dev)
+    elif p["kind"] == "contiguous":
+        out["m_indices"] = t(p["m_indices"])
+        out["D"] = torch.empty((p["M"], p["N"]), dtype=torch.bfloat16, device=dev)
+    else:
+        out["masked_m"] = t(p["masked_m"])
+        out["D"] = torch.empty((p["G"], p["max_m"], p["N"]), dtype=torch.bfloat16, device=dev)
+    return out
+
+
+def call(dg, p, d, stream=None):
+    if p["kind"] == "dense":
+        dg.dg_fp8_gemm_nt(d["A"], d["sA"], d["B"], d["sB"], d["D"], stream=stream)
+    elif p["kind"] == "contiguous":
+        dg.dg_fp8_grouped_gemm_contiguous(d["A"], d["sA"], d["B"], d["sB"], d["D"], d["m_indices"],
+                                          stream=stream)
+    else:
+        dg.dg_fp8_grouped_gemm_masked(d["A"], d["sA"], d["B"], d["sB"], d["D"], d["masked_m"],
+                                      expected_m=int(np.mean(p["masked_m"])), stream=stream)
+
+
+def time_kernel(torch, dg, p, d, steps, warmup, flush):
+    """Per-launch CUDA-event times (ms) with an L2 flush before each launch."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        call(dg, p, d)
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        call(dg, p, d)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    st = dg.dg_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {dg.dg_status_string(st)} during the benchmark")
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def time_e2e(torch, dg, p, steps, warmup, dev):
+    """Through the public API with host buffers: pinned host inputs copied in,
+    the GEMM, the output copied back -- all inside the timed region."""
+    host = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory()
+            for k, v in (("A", p["A"]), ("B", p["B"]), ("sA", gi.sa_to_kernel_layout(p["sA"])),
+                         ("sB", p["sB"]))}
+    d = to_device(p, torch, dev)
+    out_host = torch.empty(d["D"].shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for k in host:
+            d[k].copy_(host[k], non_blocking=True)
+        call(dg, p, d)
+        out_host.copy_(d["D"], non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps, h2d, d2h
+
+
+def cpu_oracle_rate(p, budget_s=10.0):
+    """The oracle as it stands on this host: FLOP/s over repeated whole-problem
+    passes (at least one) within about budget_s seconds."""
+    import oracle
+    oracle.build()
+    flop, _, _ = workload_cost(p)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.gemm_nt(p["A"], p["sA"], p["B"], p["sB"], want_f64=False)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return flop * n / dt / 1e12, oracle.num_threads(), n, dt
+
+
+# ------------------------------------------------------------------- arms
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    p = gi.make_workload(HEADLINE)
+    rows = 16  # bounded sample of the workload per step: 16 of its 128 rows
+    sub = dict(p, A=p["A"][:rows], sA=p["sA"][:rows], M=rows)
+    flop, _, _ = workload_cost(sub)
+    for _ in range(args.warmup):
+        oracle.gemm_nt(sub["A"], sub["sA"], sub["B"], sub["sB"], want_f64=False)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.gemm_nt(sub["A"], sub["sA"], sub["B"], sub["sB"], want_f64=False)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = flop / (ms * 1e-3) / 1e12
+    cores = oracle.num_threads()
+    sample = f"rows 0..{rows - 1} of the {p['M']}x{p['N']}x{p['K']} problem per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) quantised to e4m3 with 1x128 / 128x128 fp32 scales)",
+        "config": {"workload": "dense_decode M=128 N=2112 K=7168", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from moe_grouped_gemm_wt_b200 import build as b
+    if not os.path.exists(b.LIB):
+        b.build()
+    import moe_grouped_gemm_wt_b200 as dg
+    dg.load_library()
+
+    pk = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    p = gi.make_workload(HEADLINE)
+    d = to_device(p, torch, dev)
+    flop, byts, _ = workload_cost(p)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    times = time_kernel(torch, dg, p, d, args.steps, max(args.warmup, 3), flush)
+    torch.cuda.synchronize()
+    ms = sum(times) / len(times)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+
+    # per-shape sweep (every rank runs it; rank 0 reports)
+    shapes = {}
+    if not args.no_shapes:
+        for name in gi.WORKLOADS:
+            q = p if name == HEADLINE else gi.make_workload(name)
+            dq = d if name == HEADLINE else to_device(q, torch, dev)
+            tq = time_kernel(torch, dg, q, dq, max(10, min(args.steps, 30)), 3, flush)
+            mq = statistics.median(tq)
+            fq, bq, rows = workload_cost(q)
+            bound, t_roof, _ = roofline(fq, bq, pk)
+            shapes[name] = {
+                "us": mq * 1e3, "tflops": fq / (mq * 1e-3) / 1e12,
+                "bound": bound, "roofline_us": t_roof * 1e6,
+                "frac_of_roofline": t_roof / (mq * 1e-3),
+                "valid_rows": rows,
+            }
+            if name != HEADLINE:
+                del dq
+                torch.cuda.empty_cache()
+    clocks = sampler.stop()
+
+    e2e_ms, h2d, d2h = time_e2e(torch, dg, p, max(10, min(args.steps, 50)), 3, dev)
+
+    value = flop * world / (ms * 1e-3) / 1e12
+    bound, t_roof, fp8_peak = roofline(flop, byts, pk)
+    if bound == "hbm":
+        achieved = byts / (ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"]}
+    else:
+        achieved = flop / (ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp8_peak}
+    roof["traffic"] = ncu_traffic(HEADLINE)
+    roof["peak_source"] = pk["source"] + (" (fp8 = 2 x measured bf16)" if bound == "tensor" else "")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, npass, dt = cpu_oracle_rate(p, args.cpu_budget)
+        cpu = {"value": rate, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+               "sample": f"{npass} whole passes of the 128x2112x7168 problem in {dt:.1f} s"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3 (fp32 promotion, bf16 out)",
+        "data": "synthetic (seeded N(0,1) quantised to e4m3 with 1x128 / 128x128 fp32 scales)",
+        "config": {"workload": "dense_decode M=128 N=2112 K=7168",
+                   "l2": "flushed before every timed launch (512 MiB write)",
+                   "parallelism": f"replicas x{world}",
+                   "tile": dg.dg_describe_config(0, p["M"], p["N"], p["K"], 1)},
+        "roofline": roof,
+        "frac_of_roofline": t_roof / (ms * 1e-3),
+        "cpu_baseline": cpu,
+        "e2e": {"value": flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "shapes": shapes,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-shapes", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,171 @@
+/*
+ * dg_b200.h -- C ABI of the B200 (sm_100a) fine-grained-scaled FP8 GEMM.
+ *
+ * One operation, three layouts:
+ *
+ *   D[m,n] = bf16( sum_kb sA[m,kb] * sB[n/128,kb] * sum_{k in block kb} A[m,k]*B[n,k] )
+ *
+ * A and B are FP8 e4m3 ("fn": bias 7, max 448, no infinities), both K-major
+ * (the "NT" form D = A @ B.T).  There is one fp32 scale per 1x128 block of A
+ * and one per 128x128 block of B.  Each 128-wide K block is contracted on the
+ * tensor cores and its partial is then promoted into an fp32 accumulator on
+ * the CUDA cores as acc += (sA*sB) * partial.  D is bf16, rounded to nearest
+ * even once at the end.
+ *
+ * Sources (the DeepGEMM pages):
+ *  - "DeepGEMM: kernel FP8 GEMM sach va hieu qua nho scaling chi tiet"
+ *    (vi.news.hada.io/topic?id=19459):
+ *      section "Giao dien GEMM va rang buoc layout" -- D = C + A @ B.T for the
+ *      NT layout (C is absent here: D is overwritten); the LHS scale must be
+ *      TMA-aligned and transposed; fp32 scales on the Hopper path;
+ *      section "Dense va Grouped GEMM" -- contiguous grouping along M with
+ *      each expert segment aligned to the M block; masked grouping for
+ *      CUDA-graph decode, computing only the valid rows;
+ *      section "Tien ich va bien moi truong" -- set/get_num_sms,
+ *      get_mk_alignment_for_contiguous_layout, get_tma_aligned_size.
+ *  - DeepGEMM article (lqnn.cn/news/60274), section "DeepGEMM": fine-grained
+ *    scaling with two-level accumulation on the CUDA cores.
+ *  - "deepseek开源周第三天：DeepGEMM深度分析" (pxiaoer.blog): 1x128 activation
+ *    and 128x128 weight scale blocks.
+ *
+ * Conventions for every GEMM entry point:
+ *  - All tensor pointers are DEVICE pointers on the current device, owned by
+ *    the caller.  The library keeps no reference after the call returns.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream).
+ *  - Host-side validation runs first; on any failure the call returns a
+ *    non-zero status and launches nothing.
+ *  - The group metadata (m_indices, masked_m) is read only on the device, so
+ *    the calls never synchronise with the host and can be captured in a CUDA
+ *    graph after a first call on the device (which loads the module).
+ *  - Problems found on the device (bad group data, a pipeline wait that ran
+ *    past its time limit) never trap: the kernel records a code in a device
+ *    status word, leaves the affected rows untouched and returns.  Read and
+ *    clear it with dg_get_device_status().
+ *  - The library allocates no device memory for a GEMM call.
+ *  - Layout constraints: K >= 128 and K % 128 == 0; N >= 16 and N % 16 == 0;
+ *    A, B and D 16-byte aligned; sA, sB and the metadata 4-byte aligned.
+ *  - Row-major, packed (no leading-dimension arguments).
+ */
+#ifndef DG_B200_H
+#define DG_B200_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DG_OK = 0,
+    DG_ERR_INVALID_ARG = 1,    /* null pointer, bad size or count           */
+    DG_ERR_UNSUPPORTED = 2,    /* shape outside the layout constraints       */
+    DG_ERR_ALIGNMENT = 3,      /* pointer not aligned as required            */
+    DG_ERR_CUDA = 4,           /* a CUDA runtime or driver call failed       */
+    DG_ERR_TIMEOUT = 5,        /* device: a pipeline wait ran out of time    */
+    DG_ERR_BAD_GROUP_DATA = 6  /* device: m_indices / masked_m out of range  */
+} dg_status_t;
+
+/*
+ * Dense NT GEMM.
+ *   A  : [M][K]            e4m3 codes, row-major (K-major)
+ *   sA : [K/128][M_pad]    fp32, transposed and TMA-aligned:
+ *                          M_pad = dg_get_tma_aligned_size(M, 4); element
+ *                          (m, kb) at sA[kb * M_pad + m]; pad entries unread
+ *   B  : [N][K]            e4m3 codes, row-major (K-major)
+ *   sB : [ceil(N/128)][K/128] fp32, element (n/128, kb)
+ *   D  : [M][N]            bf16, written whole
+ * M == 0 is a no-op returning DG_OK.
+ */
+dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B,
+                           const float *sB, void *D, int M, int N, int K,
+                           cudaStream_t stream);
+
+/*
+ * Contiguous-layout grouped GEMM (MoE, grouping along M; N and K shared).
+ *   A         : [M_total][K]     e4m3; the rows of all groups concatenated
+ *   sA        : [K/128][M_pad]   fp32, M_pad = dg_get_tma_aligned_size(M_total, 4)
+ *   B         : [G][N][K]        e4m3, one weight matrix per group
+ *   sB        : [G][ceil(N/128)][K/128] fp32
+ *   D         : [M_total][N]     bf16
+ *   m_indices : [M_total]        int32 group of each row; a negative value
+ *                                marks a padding row
+ * Each group's segment starts on a multiple of
+ * dg_get_mk_alignment_for_contiguous_layout() rows (so M_total is a multiple
+ * of it too).  Row m is computed with group m_indices[m]; padding rows are
+ * left untouched.  A row whose index is >= G, or differs from the index of
+ * the first row of its aligned block, is left untouched and raises
+ * DG_ERR_BAD_GROUP_DATA in the device status word.
+ */
+dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA,
+                                           const void *B, const float *sB,
+                                           void *D, const int32_t *m_indices,
+                                           int M_total, int N, int K,
+                                           int num_groups, cudaStream_t stream);
+
+/*
+ * Masked-layout grouped GEMM (MoE decode under CUDA graphs).
+ *   A        : [G][max_m][K]     e4m3
+ *   sA       : [G][K/128][max_m_pad] fp32, max_m_pad = dg_get_tma_aligned_size(max_m, 4)
+ *   B        : [G][N][K]         e4m3
+ *   sB       : [G][ceil(N/128)][K/128] fp32
+ *   D        : [G][max_m][N]     bf16
+ *   masked_m : [G]               int32, valid rows of each group (device)
+ * Rows m < masked_m[g] of group g are computed; all other rows of D are left
+ * untouched.  masked_m[g] > max_m is clamped to max_m and a negative value is
+ * read as 0; both raise DG_ERR_BAD_GROUP_DATA in the device status word.
+ * expected_m is a host-side hint of the typical masked_m used to pick the
+ * tile shape (0 = use max_m); it never affects results.
+ */
+dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA,
+                                       const void *B, const float *sB, void *D,
+                                       const int32_t *masked_m, int num_groups,
+                                       int max_m, int N, int K, int expected_m,
+                                       cudaStream_t stream);
+
+/* Row alignment of each group's segment in the contiguous layout (128). */
+int dg_get_mk_alignment_for_contiguous_layout(void);
+
+/* x rounded up so that x * elem_bytes is a multiple of 16 bytes (the TMA
+ * alignment of the transposed LHS-scale rows).  elem_bytes must be 1, 2, 4,
+ * 8 or 16; returns -1 otherwise or when x < 0. */
+int dg_get_tma_aligned_size(int x, int elem_bytes);
+
+/* Caps the number of SMs the persistent kernels use (0 = all SMs of the
+ * current device).  Returns DG_ERR_INVALID_ARG for n < 0. */
+dg_status_t dg_set_num_sms(int n);
+
+/* SMs the next launch on the current device will use. */
+int dg_get_num_sms(void);
+
+/* Time limit of each pipeline wait inside the kernels, in nanoseconds
+ * (default 2e9).  A wait that runs past it makes the kernel record
+ * DG_ERR_TIMEOUT, drain its in-flight copies and return.  0 restores the
+ * default. */
+dg_status_t dg_set_wait_timeout_ns(uint64_t ns);
+
+/* Synchronises `stream`, then returns the device status word of the current
+ * device (DG_OK if no kernel reported a problem) and clears it.  The word
+ * also holds details; see dg_get_device_status_detail. */
+dg_status_t dg_get_device_status(cudaStream_t stream);
+
+/* Like dg_get_device_status but also returns the raw 32-bit word (code in
+ * bits 0-7, role in bits 8-11, stage in bits 12-19, CTA in bits 20-31) and
+ * does not clear it. */
+dg_status_t dg_get_device_status_detail(cudaStream_t stream, uint32_t *word);
+
+/* Describes the kernel configuration the library would launch for a problem
+ * (layout 0 = dense, 1 = contiguous, 2 = masked; for masked, M = expected_m
+ * and groups = G) into buf (NUL-terminated, truncated to len).  Returns the
+ * number of characters it wanted to write, or -1 on bad arguments. */
+int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf,
+                       int len);
+
+/* Human-readable name of a status code. */
+const char *dg_status_string(dg_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_B200_H */

@@ -1,0 +1,228 @@
+"""Python binding of the B200 fine-grained-scaled FP8 GEMM library.
+
+Argument marshalling only: every step of the GEMM runs in the CUDA kernels of
+``libdg_b200.so`` (see ``include/dg_b200.h`` for the C ABI).  The functions
+keep the C names and take torch tensors that already live on the GPU; there is
+no CPU path -- a CPU tensor, a missing library or a failed launch raises.
+
+Layouts (row-major, packed):
+  dense       A [M, K] e4m3, sA [K/128, M_pad] fp32, B [N, K] e4m3,
+              sB [ceil(N/128), K/128] fp32, D [M, N] bf16
+  contiguous  A [M_total, K], sA [K/128, M_total_pad], B [G, N, K],
+              sB [G, ceil(N/128), K/128], D [M_total, N], m_indices [M_total] int32
+  masked      A [G, max_m, K], sA [G, K/128, max_m_pad], B [G, N, K],
+              sB [G, ceil(N/128), K/128], D [G, max_m, N], masked_m [G] int32
+with X_pad = get_tma_aligned_size(X, 4) (the transposed, TMA-aligned LHS
+scale layout of the DeepGEMM pages, hada.io summary, section "Giao dien GEMM
+va rang buoc layout").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdg_b200.so")
+
+DG_OK = 0
+STATUS_NAMES = {
+    0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_UNSUPPORTED", 3: "DG_ERR_ALIGNMENT",
+    4: "DG_ERR_CUDA", 5: "DG_ERR_TIMEOUT", 6: "DG_ERR_BAD_GROUP_DATA",
+}
+LAYOUT_DENSE, LAYOUT_CONTIGUOUS, LAYOUT_MASKED = 0, 1, 2
+
+# Every function the header declares, with its ctypes signature.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SIGNATURES = {
+    "dg_fp8_gemm_nt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "dg_fp8_grouped_gemm_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "dg_fp8_grouped_gemm_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "dg_get_mk_alignment_for_contiguous_layout": (_I, []),
+    "dg_get_tma_aligned_size": (_I, [_I, _I]),
+    "dg_set_num_sms": (_I, [_I]),
+    "dg_get_num_sms": (_I, []),
+    "dg_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
+    "dg_get_device_status": (_I, [_P]),
+    "dg_get_device_status_detail": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "dg_describe_config": (_I, [_I, _I, _I, _I, _I, ctypes.c_char_p, _I]),
+    "dg_status_string": (ctypes.c_char_p, [_I]),
+}
+
+_lib = None
+
+
+class DGError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+def load_library(path: str | None = None):
+    """Loads libdg_b200.so (built by ``moe_grouped_gemm_wt_b200.build``)."""
+    global _lib
+    if _lib is None:
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(
+                f"CUDA library {p} is missing: run `python -m moe_grouped_gemm_wt_b200.build` "
+                "(there is no CPU fallback)")
+        lib = ctypes.CDLL(p)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != DG_OK:
+        raise DGError(fn, status)
+
+
+def _stream_handle(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str, dtypes, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+_FP8 = (torch.float8_e4m3fn, torch.uint8)
+_F32 = (torch.float32,)
+_BF16 = (torch.bfloat16,)
+_I32 = (torch.int32,)
+
+
+def get_tma_aligned_size(x: int, elem_bytes: int = 4) -> int:
+    return load_library().dg_get_tma_aligned_size(x, elem_bytes)
+
+
+def get_mk_alignment_for_contiguous_layout() -> int:
+    return load_library().dg_get_mk_alignment_for_contiguous_layout()
+
+
+def dg_get_tma_aligned_size(x: int, elem_bytes: int) -> int:
+    return get_tma_aligned_size(x, elem_bytes)
+
+
+def dg_get_mk_alignment_for_contiguous_layout() -> int:
+    return get_mk_alignment_for_contiguous_layout()
+
+
+def dg_set_num_sms(n: int) -> None:
+    _check("dg_set_num_sms", load_library().dg_set_num_sms(n))
+
+
+def dg_get_num_sms() -> int:
+    return load_library().dg_get_num_sms()
+
+
+def dg_set_wait_timeout_ns(ns: int) -> None:
+    _check("dg_set_wait_timeout_ns", load_library().dg_set_wait_timeout_ns(ns))
+
+
+def dg_get_device_status(stream=None) -> int:
+    """Synchronises the stream; returns and clears the device status code."""
+    return load_library().dg_get_device_status(_stream_handle(stream, None))
+
+
+def dg_get_device_status_detail(stream=None):
+    w = ctypes.c_uint32(0)
+    st = load_library().dg_get_device_status_detail(_stream_handle(stream, None), ctypes.byref(w))
+    return st, w.value
+
+
+def dg_describe_config(layout: int, M: int, N: int, K: int, groups: int = 1) -> str:
+    buf = ctypes.create_string_buffer(256)
+    n = load_library().dg_describe_config(layout, M, N, K, groups, buf, 256)
+    if n < 0:
+        raise ValueError("bad arguments")
+    return buf.value.decode()
+
+
+def dg_status_string(status: int) -> str:
+    return load_library().dg_status_string(status).decode()
+
+
+def dg_fp8_gemm_nt(A, sA, B, sB, D, stream=None) -> None:
+    pa = _dev(A, "A", _FP8, 2)
+    M, K = A.shape
+    N = B.shape[0] if B.dim() == 2 else -1
+    pb = _dev(B, "B", _FP8, 2)
+    if B.shape[1] != K:
+        raise ValueError("B must be [N, K]")
+    psa = _dev(sA, "sA", _F32, 2)
+    if tuple(sA.shape) != (K // 128, get_tma_aligned_size(M, 4)):
+        raise ValueError(f"sA must be [K/128, M_pad] = {(K // 128, get_tma_aligned_size(M, 4))}")
+    psb = _dev(sB, "sB", _F32, 2)
+    if tuple(sB.shape) != ((N + 127) // 128, K // 128):
+        raise ValueError("sB must be [ceil(N/128), K/128]")
+    pd = _dev(D, "D", _BF16, 2)
+    if tuple(D.shape) != (M, N):
+        raise ValueError("D must be [M, N]")
+    st = load_library().dg_fp8_gemm_nt(pa, psa, pb, psb, pd, M, N, K, _stream_handle(stream, A.device))
+    _check("dg_fp8_gemm_nt", st)
+
+
+def dg_fp8_grouped_gemm_contiguous(A, sA, B, sB, D, m_indices, stream=None) -> None:
+    pa = _dev(A, "A", _FP8, 2)
+    M, K = A.shape
+    pb = _dev(B, "B", _FP8, 3)
+    G, N, Kb = B.shape
+    if Kb != K:
+        raise ValueError("B must be [G, N, K]")
+    psa = _dev(sA, "sA", _F32, 2)
+    if tuple(sA.shape) != (K // 128, get_tma_aligned_size(M, 4)):
+        raise ValueError("sA must be [K/128, M_pad]")
+    psb = _dev(sB, "sB", _F32, 3)
+    if tuple(sB.shape) != (G, (N + 127) // 128, K // 128):
+        raise ValueError("sB must be [G, ceil(N/128), K/128]")
+    pd = _dev(D, "D", _BF16, 2)
+    if tuple(D.shape) != (M, N):
+        raise ValueError("D must be [M_total, N]")
+    pm = _dev(m_indices, "m_indices", _I32, 1)
+    if m_indices.shape[0] != M:
+        raise ValueError("m_indices must be [M_total]")
+    st = load_library().dg_fp8_grouped_gemm_contiguous(pa, psa, pb, psb, pd, pm, M, N, K, G,
+                                                       _stream_handle(stream, A.device))
+    _check("dg_fp8_grouped_gemm_contiguous", st)
+
+
+def dg_fp8_grouped_gemm_masked(A, sA, B, sB, D, masked_m, expected_m: int = 0, stream=None) -> None:
+    pa = _dev(A, "A", _FP8, 3)
+    G, max_m, K = A.shape
+    pb = _dev(B, "B", _FP8, 3)
+    if B.shape[0] != G or B.shape[2] != K:
+        raise ValueError("B must be [G, N, K]")
+    N = B.shape[1]
+    psa = _dev(sA, "sA", _F32, 3)
+    if tuple(sA.shape) != (G, K // 128, get_tma_aligned_size(max_m, 4)):
+        raise ValueError("sA must be [G, K/128, max_m_pad]")
+    psb = _dev(sB, "sB", _F32, 3)
+    if tuple(sB.shape) != (G, (N + 127) // 128, K // 128):
+        raise ValueError("sB must be [G, ceil(N/128), K/128]")
+    pd = _dev(D, "D", _BF16, 3)
+    if tuple(D.shape) != (G, max_m, N):
+        raise ValueError("D must be [G, max_m, N]")
+    pm = _dev(masked_m, "masked_m", _I32, 1)
+    if masked_m.shape[0] != G:
+        raise ValueError("masked_m must be [G]")
+    st = load_library().dg_fp8_grouped_gemm_masked(pa, psa, pb, psb, pd, pm, G, max_m, N, K,
+                                                   expected_m, _stream_handle(stream, A.device))
+    _check("dg_fp8_grouped_gemm_masked", st)

@@ -1,0 +1,433 @@
+// dg_api.cu -- host side of the C ABI declared in include/dg_b200.h:
+// argument validation, tile-shape choice, TMA descriptor encoding and kernel
+// launch.  All arithmetic of the GEMM runs in fp8_gemm_kernel.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dg_b200.h"
+#include "fp8_gemm_kernel.cuh"
+
+namespace {
+
+using dg::GemmParams;
+using dg::KernelConfig;
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+
+std::atomic<int> g_num_sms_cap{0};
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+int g_sm_count[kMaxDevices] = {0};
+
+// ------------------------------------------------------------ driver entry
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D byte matrix [rows][inner], box [box_rows][128 bytes], 128-byte swizzle.
+bool make_tmap_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                  uint32_t box_rows)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------- device
+
+int current_device()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return -1;
+    return dev;
+}
+
+int device_sm_count(int dev)
+{
+    if (dev < 0 || dev >= kMaxDevices)
+        return 0;
+    if (g_sm_count[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return 0;
+        g_sm_count[dev] = n;
+    }
+    return g_sm_count[dev];
+}
+
+int effective_sms(int dev)
+{
+    const int hw = device_sm_count(dev);
+    const int cap = g_num_sms_cap.load();
+    return (cap > 0 && cap < hw) ? cap : hw;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------- configurations
+
+// The tile widths compiled into the library.  Each has a pipeline depth that
+// fills the 227 KB of shared memory (one CTA per SM).
+struct TileChoice {
+    int bn;
+    int stages;
+};
+constexpr TileChoice kTileChoices[] = {{112, 7}, {128, 6}, {224, 5}, {256, 4}};
+
+// Deterministic choice, no autotuning (lqnn.cn article, section
+// "完全JIT设计"; non-power-of-two BLOCK_N to fill the SMs, section
+// "非对齐块大小"): the number of waves of tiles over the SMs times the time of
+// one tile, which grows with BN plus a fixed per-tile cost.
+TileChoice choose_tile(int64_t m_blocks, int N, int sms)
+{
+    TileChoice best = kTileChoices[0];
+    double best_cost = 1e300;
+    for (const TileChoice &c : kTileChoices) {
+        const int64_t n_blocks = (N + c.bn - 1) / c.bn;
+        const int64_t tiles = m_blocks * n_blocks;
+        const int64_t waves = (tiles + sms - 1) / sms;
+        // time of one tile ~ BN (MMA + promotion columns) + fixed overhead;
+        // columns beyond N in the last n-block are wasted work.
+        const double cost = static_cast<double>(waves) * (c.bn + 32);
+        if (cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && c.bn > best.bn)) {
+            best_cost = cost;
+            best = c;
+        }
+    }
+    return best;
+}
+
+int choose_raster(int num_mb)
+{
+    return num_mb < 16 ? (num_mb > 0 ? num_mb : 1) : 16;
+}
+
+template <int BN, int STAGES, int LAYOUT>
+dg_status_t launch_kernel(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+                          int grid, cudaStream_t stream)
+{
+    using Cfg = KernelConfig<BN, STAGES>;
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, LAYOUT>;
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices)
+        return DG_ERR_CUDA;
+    if (!attr_set[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::SMEM_BYTES) != cudaSuccess)
+            return DG_ERR_CUDA;
+        attr_set[dev].store(true);
+    }
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
+    if (cudaPeekAtLastError() != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DG_ERR_CUDA;
+    }
+    return DG_OK;
+}
+
+template <int LAYOUT>
+dg_status_t dispatch(const TileChoice &c, const void *A, uint64_t a_rows, const void *B,
+                     uint64_t b_rows, int K, GemmParams p, int64_t tiles_hint, int sms,
+                     cudaStream_t stream)
+{
+    CUtensorMap ta, tb;
+    if (!make_tmap_u8(&ta, A, static_cast<uint64_t>(K), a_rows, dg::kBM) ||
+        !make_tmap_u8(&tb, B, static_cast<uint64_t>(K), b_rows, static_cast<uint32_t>(c.bn)))
+        return DG_ERR_CUDA;
+    p.num_nb = (p.N + c.bn - 1) / c.bn;
+    int grid = sms;
+    if (LAYOUT != dg::kMasked) {
+        const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
+        grid = static_cast<int>(tiles < sms ? tiles : sms);
+    }
+    (void)tiles_hint;
+    if (grid <= 0)
+        return DG_OK;
+    switch (c.bn) {
+    case 112: return launch_kernel<112, 7, LAYOUT>(ta, tb, p, grid, stream);
+    case 128: return launch_kernel<128, 6, LAYOUT>(ta, tb, p, grid, stream);
+    case 224: return launch_kernel<224, 5, LAYOUT>(ta, tb, p, grid, stream);
+    case 256: return launch_kernel<256, 4, LAYOUT>(ta, tb, p, grid, stream);
+    default: return DG_ERR_UNSUPPORTED;
+    }
+}
+
+dg_status_t check_common(const void *A, const float *sA, const void *B, const float *sB,
+                         const void *D, int N, int K)
+{
+    if (!A || !sA || !B || !sB || !D)
+        return DG_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0)
+        return DG_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N % 16 != 0)
+        return DG_ERR_UNSUPPORTED;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sA, 4) ||
+        !aligned(sB, 4))
+        return DG_ERR_ALIGNMENT;
+    return DG_OK;
+}
+
+bool print_configs()
+{
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("DG_PRINT_CONFIGS");
+        v = (e && e[0] && e[0] != '0') ? 1 : 0;
+    }
+    return v == 1;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+
+extern "C" {
+
+dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B, const float *sB,
+                           void *D, int M, int N, int K, cudaStream_t stream)
+{
+    if (M < 0)
+        return DG_ERR_INVALID_ARG;
+    dg_status_t st = check_common(A, sA, B, sB, D, N, K);
+    if (st != DG_OK)
+        return st;
+    if (M == 0)
+        return DG_OK;
+    const int dev = current_device();
+    const int sms = effective_sms(dev);
+    if (sms <= 0)
+        return DG_ERR_CUDA;
+    GemmParams p{};
+    p.sA = sA;
+    p.sB = sB;
+    p.D = static_cast<__nv_bfloat16 *>(D);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = 1;
+    p.sa_ld = dg_get_tma_aligned_size(M, 4);
+    p.num_kb = K / 128;
+    p.nbn = (N + 127) / 128;
+    p.num_mb = (M + 127) / 128;
+    p.raster = choose_raster(p.num_mb);
+    p.timeout_ns = g_timeout_ns.load();
+    const TileChoice c = choose_tile(p.num_mb, N, sms);
+    if (print_configs())
+        std::fprintf(stderr, "[dg] dense M=%d N=%d K=%d -> BM=128 BN=%d stages=%d sms=%d\n", M, N,
+                     K, c.bn, c.stages, sms);
+    return dispatch<dg::kDense>(c, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), K, p,
+                                0, sms, stream);
+}
+
+dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const void *B,
+                                           const float *sB, void *D, const int32_t *m_indices,
+                                           int M_total, int N, int K, int num_groups,
+                                           cudaStream_t stream)
+{
+    if (M_total < 0 || num_groups <= 0 || !m_indices)
+        return DG_ERR_INVALID_ARG;
+    dg_status_t st = check_common(A, sA, B, sB, D, N, K);
+    if (st != DG_OK)
+        return st;
+    if (M_total % 128 != 0)
+        return DG_ERR_UNSUPPORTED;
+    if (!aligned(m_indices, 4))
+        return DG_ERR_ALIGNMENT;
+    if (M_total == 0)
+        return DG_OK;
+    if (static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF)
+        return DG_ERR_UNSUPPORTED;
+    const int dev = current_device();
+    const int sms = effective_sms(dev);
+    if (sms <= 0)
+        return DG_ERR_CUDA;
+    GemmParams p{};
+    p.sA = sA;
+    p.sB = sB;
+    p.D = static_cast<__nv_bfloat16 *>(D);
+    p.m_indices = m_indices;
+    p.M = M_total;
+    p.N = N;
+    p.K = K;
+    p.G = num_groups;
+    p.sa_ld = dg_get_tma_aligned_size(M_total, 4);
+    p.num_kb = K / 128;
+    p.nbn = (N + 127) / 128;
+    p.num_mb = M_total / 128;
+    p.raster = choose_raster(p.num_mb);
+    p.timeout_ns = g_timeout_ns.load();
+    const TileChoice c = choose_tile(p.num_mb, N, sms);
+    if (print_configs())
+        std::fprintf(stderr, "[dg] contiguous M=%d N=%d K=%d G=%d -> BM=128 BN=%d stages=%d sms=%d\n",
+                     M_total, N, K, num_groups, c.bn, c.stages, sms);
+    return dispatch<dg::kContiguous>(c, A, static_cast<uint64_t>(M_total), B,
+                                     static_cast<uint64_t>(num_groups) * N, K, p, 0, sms, stream);
+}
+
+dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const void *B,
+                                       const float *sB, void *D, const int32_t *masked_m,
+                                       int num_groups, int max_m, int N, int K, int expected_m,
+                                       cudaStream_t stream)
+{
+    if (num_groups <= 0 || max_m < 0 || expected_m < 0 || !masked_m)
+        return DG_ERR_INVALID_ARG;
+    dg_status_t st = check_common(A, sA, B, sB, D, N, K);
+    if (st != DG_OK)
+        return st;
+    if (!aligned(masked_m, 4))
+        return DG_ERR_ALIGNMENT;
+    if (max_m == 0)
+        return DG_OK;
+    if (static_cast<int64_t>(num_groups) * max_m > 0x7FFFFFFF ||
+        static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF)
+        return DG_ERR_UNSUPPORTED;
+    const int dev = current_device();
+    const int sms = effective_sms(dev);
+    if (sms <= 0)
+        return DG_ERR_CUDA;
+    GemmParams p{};
+    p.sA = sA;
+    p.sB = sB;
+    p.D = static_cast<__nv_bfloat16 *>(D);
+    p.masked_m = masked_m;
+    p.M = max_m;
+    p.N = N;
+    p.K = K;
+    p.G = num_groups;
+    p.sa_ld = dg_get_tma_aligned_size(max_m, 4);
+    p.num_kb = K / 128;
+    p.nbn = (N + 127) / 128;
+    p.num_mb = (max_m + 127) / 128;
+    p.raster = 1;
+    p.timeout_ns = g_timeout_ns.load();
+    const int em = (expected_m > 0 && expected_m < max_m) ? expected_m : max_m;
+    const TileChoice c = choose_tile(static_cast<int64_t>(num_groups) * ((em + 127) / 128), N, sms);
+    if (print_configs())
+        std::fprintf(stderr,
+                     "[dg] masked G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=128 BN=%d stages=%d sms=%d\n",
+                     num_groups, max_m, em, N, K, c.bn, c.stages, sms);
+    return dispatch<dg::kMasked>(c, A, static_cast<uint64_t>(num_groups) * max_m, B,
+                                 static_cast<uint64_t>(num_groups) * N, K, p, 0, sms, stream);
+}
+
+int dg_get_mk_alignment_for_contiguous_layout(void) { return 128; }
+
+int dg_get_tma_aligned_size(int x, int elem_bytes)
+{
+    if (x < 0 || !(elem_bytes == 1 || elem_bytes == 2 || elem_bytes == 4 || elem_bytes == 8 ||
+                   elem_bytes == 16))
+        return -1;
+    const int per = 16 / elem_bytes;
+    return (x + per - 1) / per * per;
+}
+
+dg_status_t dg_set_num_sms(int n)
+{
+    if (n < 0)
+        return DG_ERR_INVALID_ARG;
+    g_num_sms_cap.store(n);
+    return DG_OK;
+}
+
+int dg_get_num_sms(void) { return effective_sms(current_device()); }
+
+dg_status_t dg_set_wait_timeout_ns(uint64_t ns)
+{
+    g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
+    return DG_OK;
+}
+
+dg_status_t dg_get_device_status_detail(cudaStream_t stream, uint32_t *word)
+{
+    if (!word)
+        return DG_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
+        return DG_ERR_CUDA;
+    unsigned int w = 0;
+    if (cudaMemcpyFromSymbol(&w, dg::g_status_word, sizeof(w)) != cudaSuccess)
+        return DG_ERR_CUDA;
+    *word = w;
+    return static_cast<dg_status_t>(w & 0xFF);
+}
+
+dg_status_t dg_get_device_status(cudaStream_t stream)
+{
+    uint32_t w = 0;
+    dg_status_t st = dg_get_device_status_detail(stream, &w);
+    if (st == DG_ERR_CUDA || st == DG_ERR_INVALID_ARG)
+        return st;
+    if (w != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(dg::g_status_word, &zero, sizeof(zero)) != cudaSuccess)
+            return DG_ERR_CUDA;
+    }
+    return static_cast<dg_status_t>(w & 0xFF);
+}
+
+int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, int len)
+{
+    if (layout < 0 || layout > 2 || M < 0 || N <= 0 || K <= 0 || groups <= 0 || (len > 0 && !buf))
+        return -1;
+    // Without a device (host-only use) the SM cap alone decides, else 148.
+    const int dev = current_device();
+    int sms = effective_sms(dev);
+    if (sms <= 0)
+        sms = g_num_sms_cap.load() > 0 ? g_num_sms_cap.load() : 148;
+    int64_t m_blocks = (M + 127) / 128;
+    if (layout == 2)
+        m_blocks *= groups;
+    const TileChoice c = choose_tile(m_blocks, N, sms);
+    return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
+                         "layout=%d BM=128 BN=%d BK=128 stages=%d sms=%d m_blocks=%lld n_blocks=%d",
+                         layout, c.bn, c.stages, sms, static_cast<long long>(m_blocks),
+                         (N + c.bn - 1) / c.bn);
+}
+
+const char *dg_status_string(dg_status_t status)
+{
+    switch (status) {
+    case DG_OK: return "DG_OK";
+    case DG_ERR_INVALID_ARG: return "DG_ERR_INVALID_ARG";
+    case DG_ERR_UNSUPPORTED: return "DG_ERR_UNSUPPORTED";
+    case DG_ERR_ALIGNMENT: return "DG_ERR_ALIGNMENT";
+    case DG_ERR_CUDA: return "DG_ERR_CUDA";
+    case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT";
+    case DG_ERR_BAD_GROUP_DATA: return "DG_ERR_BAD_GROUP_DATA";
+    }
+    return "DG_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,103 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every function the
+header declares, and its host logic (validation, alignment helpers, status
+names, tile choice) behaves as documented -- no GPU compute is called."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from moe_grouped_gemm_wt_b200 import build as b
+    b.build()
+    import moe_grouped_gemm_wt_b200 as dg
+    return dg.load_library()
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(dg_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert "dg_fp8_gemm_nt" in names and len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_binding_covers_header():
+    import moe_grouped_gemm_wt_b200 as dg
+    for n in _declared_functions():
+        assert n in dg._SIGNATURES, n
+        assert callable(getattr(dg, n)), n
+
+
+def test_host_helpers(lib):
+    assert lib.dg_get_mk_alignment_for_contiguous_layout() == 128
+    assert lib.dg_get_tma_aligned_size(1, 4) == 4
+    assert lib.dg_get_tma_aligned_size(130, 4) == 132
+    assert lib.dg_get_tma_aligned_size(17, 1) == 32
+    assert lib.dg_get_tma_aligned_size(5, 3) == -1
+    assert lib.dg_get_tma_aligned_size(-1, 4) == -1
+    assert lib.dg_status_string(0) == b"DG_OK"
+    assert lib.dg_status_string(5) == b"DG_ERR_TIMEOUT"
+    assert lib.dg_set_num_sms(-1) == 1
+    assert lib.dg_set_wait_timeout_ns(0) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("M,N,K,expect", [
+    (128, 256, 500, 2),    # K not a multiple of 128
+    (128, 250, 512, 2),    # N not a multiple of 16
+    (-1, 256, 512, 1),
+    (128, 0, 512, 1),
+])
+def test_dense_validation(lib, M, N, K, expect):
+    st = lib.dg_fp8_gemm_nt(FAKE, FAKE, FAKE, FAKE, FAKE, M, N, K, None)
+    assert st == expect
+
+
+def test_null_and_alignment(lib):
+    assert lib.dg_fp8_gemm_nt(None, FAKE, FAKE, FAKE, FAKE, 128, 256, 512, None) == 1
+    odd = ctypes.c_void_p(0x10008)
+    assert lib.dg_fp8_gemm_nt(odd, FAKE, FAKE, FAKE, FAKE, 128, 256, 512, None) == 3
+    # contiguous: M_total must be a multiple of the 128-row alignment
+    assert lib.dg_fp8_grouped_gemm_contiguous(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 200, 256, 512, 2, None) == 2
+    assert lib.dg_fp8_grouped_gemm_contiguous(FAKE, FAKE, FAKE, FAKE, FAKE, None, 256, 256, 512, 2, None) == 1
+    # masked: bad counts
+    assert lib.dg_fp8_grouped_gemm_masked(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 256, 512, 0, None) == 1
+    assert lib.dg_fp8_grouped_gemm_masked(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, -1, 256, 512, 0, None) == 1
+    # empty problems are no-ops
+    assert lib.dg_fp8_gemm_nt(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 512, None) == 0
+
+
+def test_sm_fill_example_from_pages(lib):
+    """The unaligned-block-size example of the DeepGEMM article (lqnn.cn,
+    section 非对齐块大小): M=256, N=7168 on 132 SMs -- 128x128 tiles occupy
+    112 SMs, 128x112 tiles occupy 128, so BLOCK_N=112 is the better choice."""
+    ex = json.load(open(os.path.join(ROOT, "tests", "golden", "sm_fill_example.json")))
+    assert lib.dg_set_num_sms(ex["num_sms"]) == 0
+    try:
+        buf = ctypes.create_string_buffer(256)
+        lib.dg_describe_config(0, ex["M"], ex["N"], 7168, 1, buf, 256)
+        desc = dict(kv.split("=") for kv in buf.value.decode().split())
+        assert int(desc["BN"]) == ex["chosen_block_n"]
+        m_blocks = ex["M"] // 128
+        for bn, used in ex["sms_used_by_block_n"].items():
+            tiles = m_blocks * ((ex["N"] + int(bn) - 1) // int(bn))
+            assert min(tiles, ex["num_sms"]) == used
+    finally:
+        lib.dg_set_num_sms(0)
