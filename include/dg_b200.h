@@ -43,7 +43,7 @@
  *    clear it with dg_get_device_status().
  *  - The library allocates no device memory for a GEMM call.
  *  - Layout constraints: K >= 128 and K % 128 == 0; N >= 16 and N % 16 == 0;
- *    A, B and D 16-byte aligned; sA, sB and the metadata 4-byte aligned.
+ *    A, B, D and sA 16-byte aligned; sB and the metadata 4-byte aligned.
  *  - Row-major, packed (no leading-dimension arguments).
  */
 #ifndef DG_B200_H

@@ -47,20 +47,39 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 2-D byte matrix [rows][inner], box [box_rows][128 bytes], 128-byte swizzle.
-bool make_tmap_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
-                  uint32_t box_rows)
+// An e4m3 operand [rows][K] viewed in 3-D as (byte within a 128-wide K
+// block, row, K block), so that one box of [ks][box_rows][128 bytes] fetches
+// ks consecutive K blocks of box_rows rows, each block a 128-byte-swizzled
+// K-major tile.
+bool make_tmap_operand(CUtensorMap *map, const void *base, uint64_t K, uint64_t rows,
+                       uint32_t box_rows, uint32_t ks)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[3] = {128, rows, K / 128};
+    cuuint64_t strides[2] = {K, 128};
+    cuuint32_t box[3] = {128, box_rows, ks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D bf16 matrix [rows][inner] (the output), box [box_rows][box_inner].
+bool make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                    uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc)
         return false;
     cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner};
-    cuuint32_t box[2] = {128, box_rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -103,15 +122,31 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 struct TileChoice {
     int bn;
     int stages;
+    int ks;  // 128-wide K blocks per pipeline stage
 };
-constexpr TileChoice kTileChoices[] = {{112, 7}, {128, 6}, {224, 5}, {256, 4}};
+constexpr TileChoice kTileChoices[] = {{112, 3, 2}, {128, 5, 1}, {224, 2, 2}, {256, 3, 1}};
 
 // Deterministic choice, no autotuning (lqnn.cn article, section
 // "完全JIT设计"; non-power-of-two BLOCK_N to fill the SMs, section
 // "非对齐块大小"): the number of waves of tiles over the SMs times the time of
 // one tile, which grows with BN plus a fixed per-tile cost.
+// DG_FORCE_BLOCK_N=<n> pins the tile width to one of the compiled choices
+// (read once; for tuning sweeps).
+int forced_block_n()
+{
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("DG_FORCE_BLOCK_N");
+        v = e ? std::atoi(e) : 0;
+    }
+    return v;
+}
+
 TileChoice choose_tile(int64_t m_blocks, int N, int sms)
 {
+    for (const TileChoice &c : kTileChoices)
+        if (c.bn == forced_block_n())
+            return c;
     TileChoice best = kTileChoices[0];
     double best_cost = 1e300;
     for (const TileChoice &c : kTileChoices) {
@@ -134,12 +169,30 @@ int choose_raster(int num_mb)
     return num_mb < 16 ? (num_mb > 0 ? num_mb : 1) : 16;
 }
 
-template <int BN, int STAGES, int LAYOUT>
-dg_status_t launch_kernel(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
-                          int grid, cudaStream_t stream)
+template <int BN, int STAGES, int KS, int LAYOUT>
+dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
+                          const GemmParams &p, int grid, cudaStream_t stream)
 {
-    using Cfg = KernelConfig<BN, STAGES>;
-    auto kern = dg::fp8_gemm_kernel<BN, STAGES, LAYOUT>;
+    using Cfg = KernelConfig<BN, STAGES, KS>;
+    CUtensorMap ta, tb;
+    if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
+        !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, BN, KS))
+        return DG_ERR_CUDA;
+    const uint64_t d_rows = a_rows;
+    // output boxes of 32 rows: 64 columns with 128-byte swizzle, and the
+    // warpgroup's remainder columns unswizzled
+    CUtensorMap td64, tdrem;
+    if (!make_tmap_bf16(&td64, p.D, static_cast<uint64_t>(p.N), d_rows, 64, dg::kBM,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return DG_ERR_CUDA;
+    if (Cfg::EPI_REM > 0) {
+        if (!make_tmap_bf16(&tdrem, p.D, static_cast<uint64_t>(p.N), d_rows, Cfg::EPI_REM, dg::kBM,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+            return DG_ERR_CUDA;
+    } else {
+        tdrem = td64;
+    }
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices)
@@ -150,7 +203,7 @@ dg_status_t launch_kernel(const CUtensorMap &ta, const CUtensorMap &tb, const Ge
             return DG_ERR_CUDA;
         attr_set[dev].store(true);
     }
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, td64, tdrem, p);
     if (cudaPeekAtLastError() != cudaSuccess) {
         (void)cudaGetLastError();
         return DG_ERR_CUDA;
@@ -160,29 +213,25 @@ dg_status_t launch_kernel(const CUtensorMap &ta, const CUtensorMap &tb, const Ge
 
 template <int LAYOUT>
 dg_status_t dispatch(const TileChoice &c, const void *A, uint64_t a_rows, const void *B,
-                     uint64_t b_rows, int K, GemmParams p, int64_t tiles_hint, int sms,
-                     cudaStream_t stream)
+                     uint64_t b_rows, GemmParams p, int sms, cudaStream_t stream)
 {
-    CUtensorMap ta, tb;
-    if (!make_tmap_u8(&ta, A, static_cast<uint64_t>(K), a_rows, dg::kBM) ||
-        !make_tmap_u8(&tb, B, static_cast<uint64_t>(K), b_rows, static_cast<uint32_t>(c.bn)))
-        return DG_ERR_CUDA;
     p.num_nb = (p.N + c.bn - 1) / c.bn;
     int grid = sms;
     if (LAYOUT != dg::kMasked) {
         const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
         grid = static_cast<int>(tiles < sms ? tiles : sms);
     }
-    (void)tiles_hint;
     if (grid <= 0)
         return DG_OK;
-    switch (c.bn) {
-    case 112: return launch_kernel<112, 7, LAYOUT>(ta, tb, p, grid, stream);
-    case 128: return launch_kernel<128, 6, LAYOUT>(ta, tb, p, grid, stream);
-    case 224: return launch_kernel<224, 5, LAYOUT>(ta, tb, p, grid, stream);
-    case 256: return launch_kernel<256, 4, LAYOUT>(ta, tb, p, grid, stream);
-    default: return DG_ERR_UNSUPPORTED;
-    }
+#define DG_TILE_CASE(BN_, ST_, KS_)                                                         \
+    if (c.bn == BN_ && c.stages == ST_ && c.ks == KS_)                                       \
+        return launch_kernel<BN_, ST_, KS_, LAYOUT>(A, a_rows, B, b_rows, p, grid, stream);
+    DG_TILE_CASE(112, 3, 2)
+    DG_TILE_CASE(128, 5, 1)
+    DG_TILE_CASE(224, 2, 2)
+    DG_TILE_CASE(256, 3, 1)
+#undef DG_TILE_CASE
+    return DG_ERR_UNSUPPORTED;
 }
 
 dg_status_t check_common(const void *A, const float *sA, const void *B, const float *sB,
@@ -194,7 +243,7 @@ dg_status_t check_common(const void *A, const float *sA, const void *B, const fl
         return DG_ERR_INVALID_ARG;
     if (K % 128 != 0 || N % 16 != 0)
         return DG_ERR_UNSUPPORTED;
-    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sA, 4) ||
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sA, 16) ||
         !aligned(sB, 4))
         return DG_ERR_ALIGNMENT;
     return DG_OK;
@@ -246,10 +295,10 @@ dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B, const 
     p.timeout_ns = g_timeout_ns.load();
     const TileChoice c = choose_tile(p.num_mb, N, sms);
     if (print_configs())
-        std::fprintf(stderr, "[dg] dense M=%d N=%d K=%d -> BM=128 BN=%d stages=%d sms=%d\n", M, N,
-                     K, c.bn, c.stages, sms);
-    return dispatch<dg::kDense>(c, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), K, p,
-                                0, sms, stream);
+        std::fprintf(stderr, "[dg] dense M=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n", M, N,
+                     K, c.bn, c.stages, c.ks, sms);
+    return dispatch<dg::kDense>(c, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), p, sms,
+                                stream);
 }
 
 dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const void *B,
@@ -294,7 +343,7 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const
         std::fprintf(stderr, "[dg] contiguous M=%d N=%d K=%d G=%d -> BM=128 BN=%d stages=%d sms=%d\n",
                      M_total, N, K, num_groups, c.bn, c.stages, sms);
     return dispatch<dg::kContiguous>(c, A, static_cast<uint64_t>(M_total), B,
-                                     static_cast<uint64_t>(num_groups) * N, K, p, 0, sms, stream);
+                                     static_cast<uint64_t>(num_groups) * N, p, sms, stream);
 }
 
 dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const void *B,
@@ -340,7 +389,7 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const voi
                      "[dg] masked G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=128 BN=%d stages=%d sms=%d\n",
                      num_groups, max_m, em, N, K, c.bn, c.stages, sms);
     return dispatch<dg::kMasked>(c, A, static_cast<uint64_t>(num_groups) * max_m, B,
-                                 static_cast<uint64_t>(num_groups) * N, K, p, 0, sms, stream);
+                                 static_cast<uint64_t>(num_groups) * N, p, sms, stream);
 }
 
 int dg_get_mk_alignment_for_contiguous_layout(void) { return 128; }
@@ -411,8 +460,8 @@ int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, i
         m_blocks *= groups;
     const TileChoice c = choose_tile(m_blocks, N, sms);
     return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
-                         "layout=%d BM=128 BN=%d BK=128 stages=%d sms=%d m_blocks=%lld n_blocks=%d",
-                         layout, c.bn, c.stages, sms, static_cast<long long>(m_blocks),
+                         "layout=%d BM=128 BN=%d BK=128 stages=%d ks=%d sms=%d m_blocks=%lld n_blocks=%d",
+                         layout, c.bn, c.stages, c.ks, sms, static_cast<long long>(m_blocks),
                          (N + c.bn - 1) / c.bn);
 }
 

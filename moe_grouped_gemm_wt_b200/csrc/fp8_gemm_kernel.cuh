@@ -12,22 +12,33 @@
 // compile-time constants (section "完全JIT设计").
 //
 // B200 design of one CTA (one per SM, persistent over tiles of 128 x BN):
-//   warp P (producer)  : TMA loads of the A tile (128 x 128 e4m3) and the
-//                        B tile (BN x 128 e4m3) of each K block into a
-//                        STAGES-deep shared-memory ring (mbarrier full/empty).
+//   warp P (producer)  : per stage of KS K blocks, one 3-D TMA box of A
+//                        (KS x 128 x 128 e4m3) and one of B (KS x BN x 128),
+//                        plus cp.async copies of the 128 LHS scales and the
+//                        (at most three) weight-block scales of each K block,
+//                        into a STAGES-deep shared-memory ring; all land on
+//                        the stage's "full" mbarrier (lqnn.cn article,
+//                        section "Hopper TMA特性": TMA for the operands; the
+//                        scales take the LSU path because each TMA
+//                        instruction costs the SM's TMA engine a roughly
+//                        fixed time, whatever its size).
 //   warp M (MMA)       : 4 x tcgen05.mma kind::f8f6f4 (K = 32 each) per K
-//                        block into one of two TMEM partial buffers, then
+//                        block into one of NBUF (2..4) TMEM partial buffers,
+//                        issued by one elected lane of a warp-uniform loop
+//                        so the descriptors stay uniform, then
 //                        tcgen05.commit to free the smem stage and to hand
 //                        the partial to the promotion warps.
-//   promotion warps    : 1 or 2 warpgroups (BN <= 128: one; otherwise two,
-//                        splitting the columns).  Thread t of a warpgroup owns
-//                        tile row t (= TMEM lane t).  Per K block it loads its
-//                        row's partial from TMEM, frees the buffer, and does
-//                        acc = fma(partial, sA*sB, acc) in registers.  The
-//                        scales are read with plain (cached) loads one block
-//                        ahead.  After the last block it rounds to bf16 and
-//                        stores its row segment.
-// The MMA of block kb+1 runs while block kb is being promoted (double TMEM),
+//   promotion warps    : two warpgroups splitting the tile's columns.
+//                        Thread t of a warpgroup owns tile row t (= TMEM
+//                        lane t).  Per K block it loads its row's partial
+//                        from TMEM, frees the buffer, and does
+//                        acc = fma(partial, sA*sB, acc) in registers, with
+//                        the scales read from the stage in shared memory
+//                        (released through a per-stage "scales read"
+//                        barrier, since the MMA frees the operand tiles
+//                        earlier).  After the last block it rounds to bf16
+//                        and stores its row segment.
+// The MMAs of blocks kb+1 .. kb+NBUF-1 run while block kb is being promoted,
 // and the next tile's first MMAs run under the previous tile's epilogue.
 //
 // Every mbarrier wait is bounded in time: on expiry the waiting role records
@@ -195,64 +206,128 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
 
 // ------------------------------------------------------------------ config
 
-template <int BN_, int STAGES_>
+// BN: tile width; STAGES: shared-memory ring depth; KS: 128-wide K blocks per
+// stage (one 3-D TMA box per operand carries all KS blocks -- the TMA engine
+// costs a roughly fixed time per instruction, so bigger boxes move more).
+template <int BN_, int STAGES_, int KS_>
 struct KernelConfig {
     static constexpr int BN = BN_;
     static constexpr int STAGES = STAGES_;
-    static constexpr int NUM_WG = BN > 128 ? 2 : 1;
+    static constexpr int KS = KS_;
+    // Two promotion warpgroups split the tile's columns; thread t of each
+    // owns tile row t.
+    static constexpr int NUM_WG = 2;
     static constexpr int BN_WG = BN / NUM_WG;
+    // TMEM is read in rounds of at most RMAX columns: a warpgroup with at
+    // most 64 columns pulls its whole partial in one round and frees the
+    // buffer before any arithmetic.
+    static constexpr int RMAX = BN_WG <= 64 ? BN_WG : 32;
     static constexpr int NUM_PROMO_WARPS = 4 * NUM_WG;
     static constexpr int PRODUCER_WARP = NUM_PROMO_WARPS;
     static constexpr int MMA_WARP = NUM_PROMO_WARPS + 1;
     static constexpr int THREADS = (NUM_PROMO_WARPS + 2) * 32;
-    static constexpr int A_BYTES = kBM * kBK;
-    static constexpr int B_BYTES = BN * kBK;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int ACC_STRIDE = BN <= 128 ? 128 : 256;  // TMEM columns per buffer
-    static constexpr int TMEM_COLS = 2 * ACC_STRIDE;
-    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4) + 16;
-    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + BAR_BYTES;
+    static constexpr int A_BYTES = kBM * kBK;  // one K block of A
+    static constexpr int B_BYTES = BN * kBK;   // one K block of B
+    static constexpr int STAGE_BYTES = KS * (A_BYTES + B_BYTES);
+    static constexpr int SA_BYTES = KS * kBM * 4;  // LHS scales of a stage
+    static constexpr int SB_BYTES = KS * 16;       // up to 3 weight-block scales per K block
+    // TMEM: NBUF partial buffers of ACC_STRIDE columns (<= 512 in total), so
+    // the MMA can run NBUF-1 K blocks ahead of the promotion.
+    static constexpr int ACC_STRIDE = (BN + 31) / 32 * 32;
+    static constexpr int NBUF = (512 / ACC_STRIDE) < 4 ? (512 / ACC_STRIDE) : 4;
+    static constexpr int TMEM_COLS = NBUF * ACC_STRIDE <= 256 ? 256 : 512;
+    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 2 * NBUF) + 16;
+    // Epilogue: each promotion warpgroup stages its 128 rows of the output in
+    // shared memory one box at a time and TMA-stores it: boxes of 64 columns
+    // (128-byte rows, 128-byte swizzle) and one remainder box.
+    static constexpr int EPI_FULL_BOXES = BN_WG / 64;
+    static constexpr int EPI_REM = BN_WG % 64;
+    static constexpr int EPI_WG_BYTES = kBM * 128;  // 128 rows x 128 bytes
+    static constexpr int PIPE_BYTES = STAGES * (STAGE_BYTES + SA_BYTES + SB_BYTES);
+    static constexpr int EPI_OFFSET = (PIPE_BYTES + BAR_BYTES + 1023) / 1024 * 1024;
+    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + EPI_OFFSET + NUM_WG * EPI_WG_BYTES;
 
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128: multiple of 16, <= 256");
-    static_assert(BN_WG % 16 == 0, "promotion columns per warpgroup must be a multiple of 16");
-    static_assert(BN_WG <= 128, "a warpgroup's column range must fit one 128-wide sB block pair");
-    static_assert(B_BYTES % 1024 == 0, "B stage must keep 1024-byte swizzle atoms aligned");
+    static_assert(BN_WG % 8 == 0, "promotion columns per warpgroup must be a multiple of 8");
+    static_assert(BN_WG <= 128, "a warpgroup's columns must span at most two 128-wide sB blocks");
+    static_assert(NBUF >= 2, "double-buffered TMEM at least");
+    static_assert(B_BYTES % 1024 == 0, "B tiles must keep 1024-byte swizzle atoms aligned");
+    static_assert(KS >= 1 && KS <= 4, "K blocks per stage");
+    static_assert(EPI_REM % 8 == 0, "remainder box must be whole 16-byte chunks");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
+// Loads COLS (multiple of 8, may be 0) consecutive TMEM columns of this
+// warp's 32 lanes into r[0..COLS).
+template <int COLS>
+__device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *r)
+{
+#pragma unroll
+    for (int q = 0; q < COLS; q += 16) {
+        if (q + 16 <= COLS)
+            tmem_ld_32x32b_x16(taddr + q, *reinterpret_cast<uint32_t(*)[16]>(r + q));
+        else
+            tmem_ld_32x32b_x8(taddr + q, *reinterpret_cast<uint32_t(*)[8]>(r + q));
+    }
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float *v)
+{
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]);
+    __nv_bfloat162 h3 = __floats2bfloat162_rn(v[6], v[7]);
+    uint4 u;
+    u.x = *reinterpret_cast<uint32_t *>(&h0);
+    u.y = *reinterpret_cast<uint32_t *>(&h1);
+    u.z = *reinterpret_cast<uint32_t *>(&h2);
+    u.w = *reinterpret_cast<uint32_t *>(&h3);
+    return u;
+}
+
 // ------------------------------------------------------------------ kernel
 
-template <int BN, int STAGES, int LAYOUT>
-__global__ void __launch_bounds__(KernelConfig<BN, STAGES>::THREADS, 1)
+template <int BN, int STAGES, int KS, int LAYOUT>
+__global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                    const __grid_constant__ CUtensorMap tmap_b, const GemmParams p)
+                    const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_d64,
+                    const __grid_constant__ CUtensorMap tmap_drem, const GemmParams p)
 {
-    using Cfg = KernelConfig<BN, STAGES>;
+    using Cfg = KernelConfig<BN, STAGES, KS>;
     constexpr int BN_WG = Cfg::BN_WG;
-    constexpr int CHUNKS = BN_WG / 16;
+    constexpr int RMAX = Cfg::RMAX;
+    constexpr int NBUF = Cfg::NBUF;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t *a_tiles = smem;
-    uint8_t *b_tiles = smem + STAGES * Cfg::A_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * Cfg::STAGE_BYTES);
-    uint64_t *full_bar = bars;
-    uint64_t *empty_bar = bars + STAGES;
-    uint64_t *tfull_bar = bars + 2 * STAGES;
-    uint64_t *tempty_bar = bars + 2 * STAGES + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
+    uint8_t *a_tiles = smem;                                   // [STAGES*KS][128][128 B]
+    uint8_t *b_tiles = smem + STAGES * KS * Cfg::A_BYTES;      // [STAGES*KS][BN][128 B]
+    float *sa_tiles = reinterpret_cast<float *>(smem + STAGES * Cfg::STAGE_BYTES);  // [STAGES*KS][128]
+    float *sb_tiles = sa_tiles + STAGES * KS * kBM;            // [STAGES*KS][4]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sb_tiles + STAGES * KS * 4);
+    uint64_t *full_bar = bars;                 // stage landed (TMA bytes + scale copies)
+    uint64_t *empty_bar = bars + STAGES;       // MMAs of the stage done (operand tiles free)
+    uint64_t *sread_bar = bars + 2 * STAGES;   // promotion warps have read the stage's scales
+    uint64_t *tfull_bar = bars + 3 * STAGES;   // TMEM partial buffer written
+    uint64_t *tempty_bar = bars + 3 * STAGES + NBUF;  // TMEM partial buffer read out
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 2 * NBUF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    uint8_t *epi_stage = smem + Cfg::EPI_OFFSET;  // 1024-byte aligned, one buffer per warpgroup
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
 
     if (warp == Cfg::PRODUCER_WARP && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_addr(full_bar + s), 1);
+            // full: the elected producer lane's expect-tx arrival plus one
+            // cp.async arrival from each of the 32 producer lanes
+            mbar_init(smem_addr(full_bar + s), 1 + 32);
             mbar_init(smem_addr(empty_bar + s), 1);
+            mbar_init(smem_addr(sread_bar + s), Cfg::NUM_PROMO_WARPS);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NBUF; ++b) {
             mbar_init(smem_addr(tfull_bar + b), 1);
             mbar_init(smem_addr(tempty_bar + b), Cfg::NUM_PROMO_WARPS);
         }
@@ -260,6 +335,10 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES>::THREADS, 1)
         fence_barrier_init();
         tma_prefetch_desc(&tmap_a);
         tma_prefetch_desc(&tmap_b);
+        if (Cfg::EPI_FULL_BOXES > 0)
+            tma_prefetch_desc(&tmap_d64);
+        if (Cfg::EPI_REM > 0)
+            tma_prefetch_desc(&tmap_drem);
     }
     if (warp == Cfg::MMA_WARP) {
         tmem_alloc(smem_addr(tmem_slot), Cfg::TMEM_COLS);
@@ -273,36 +352,69 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES>::THREADS, 1)
 
     if (warp == Cfg::PRODUCER_WARP) {
         // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            TileScheduler<LAYOUT> sched(p);
-            TileCoord tc;
-            uint32_t stage = 0, phase = 0;
-            uint32_t issued = 0;
-            bool ok = true;
-            while (ok && sched.next(tc, true)) {
-                const int a_row = (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * kBM;
-                const int b_row = tc.g * p.N + tc.nb * BN;
-                for (int kb = 0; kb < p.num_kb; ++kb) {
-                    if (!wait_bounded(smem_addr(empty_bar + stage), phase ^ 1, tmo, abort_flag,
-                                      kRoleProducer, stage, true)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = smem_addr(full_bar + stage);
+        // The whole warp runs the loop (uniform control flow).  One elected
+        // lane issues the two operand boxes of a stage; every lane copies a
+        // 16-byte piece of each K block's LHS scales, and lanes 0-2 copy the
+        // weight-block scales, all landing on the stage's full barrier.
+        TileScheduler<LAYOUT> sched(p);
+        TileCoord tc;
+        uint32_t stage = 0, phase = 0;
+        uint32_t issued = 0;
+        bool ok = true;
+        while (ok && sched.next(tc, lane == 0)) {
+            const int a_row = (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * kBM;
+            const int b_row = tc.g * p.N + tc.nb * BN;
+            const int m0 = tc.mb * kBM;
+            const float *sa_base = p.sA +
+                                   (LAYOUT == kMasked ? static_cast<size_t>(tc.g) * p.num_kb * p.sa_ld : 0) +
+                                   m0 + 4 * lane;
+            const bool sa_lane_ok = m0 + 4 * lane < p.sa_ld;
+            // weight-block scales of the (up to three) 128-row blocks under
+            // this tile's columns (lane j copies block nb_first + j, clamped)
+            const int nb_first = (tc.nb * BN) / 128;
+            const float *sb_src = p.sB + (static_cast<size_t>(tc.g) * p.nbn +
+                                          min(nb_first + (lane < 3 ? lane : 0), p.nbn - 1)) * p.num_kb;
+            for (int kb0 = 0; kb0 < p.num_kb; kb0 += KS) {
+                if (!warp_wait_bounded(smem_addr(empty_bar + stage), phase ^ 1, tmo, abort_flag,
+                                       kRoleProducer, stage) ||
+                    !warp_wait_bounded(smem_addr(sread_bar + stage), phase ^ 1, tmo, abort_flag,
+                                       kRoleProducer, 64 + stage)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = smem_addr(full_bar + stage);
+                if (elect_one()) {
                     mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
-                    tma_load_2d(smem_addr(a_tiles + stage * Cfg::A_BYTES), &tmap_a, fb, kb * kBK,
-                                a_row);
-                    tma_load_2d(smem_addr(b_tiles + stage * Cfg::B_BYTES), &tmap_b, fb, kb * kBK,
-                                b_row);
-                    ++issued;
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
+                    tma_load_3d(smem_addr(a_tiles + stage * KS * Cfg::A_BYTES), &tmap_a, fb, 0,
+                                a_row, kb0);
+                    tma_load_3d(smem_addr(b_tiles + stage * KS * Cfg::B_BYTES), &tmap_b, fb, 0,
+                                b_row, kb0);
+                }
+#pragma unroll
+                for (int q = 0; q < KS; ++q) {
+                    const int kb = kb0 + q;
+                    const bool in_k = kb < p.num_kb;
+                    const bool sa_ok = in_k && sa_lane_ok;
+                    cp_async_16(smem_addr(sa_tiles + (stage * KS + q) * kBM) + 16 * lane,
+                                sa_ok ? static_cast<const void *>(sa_base + static_cast<size_t>(kb) * p.sa_ld)
+                                      : static_cast<const void *>(p.sA),
+                                sa_ok ? 16u : 0u);
+                    if (lane < 3)
+                        cp_async_4(smem_addr(sb_tiles + (stage * KS + q) * 4) + 4 * lane,
+                                   sb_src + (in_k ? kb : p.num_kb - 1));
+                }
+                cp_async_mbar_arrive_noinc(fb);
+                __syncwarp();
+                ++issued;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
                 }
             }
-            // Drain: the last min(STAGES, issued) loads must have landed
-            // before the CTA may exit (always true on the normal path).
+        }
+        // Drain: the last min(STAGES, issued) stages must have landed before
+        // the CTA may exit (always true on the normal path).
+        if (lane == 0) {
             const uint32_t first = issued > STAGES ? issued - STAGES : 0;
             for (uint32_t i = first; i < issued; ++i)
                 wait_bounded(smem_addr(full_bar + i % STAGES), (i / STAGES) & 1, tmo, abort_flag,
@@ -311,47 +423,64 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES>::THREADS, 1)
         __syncwarp();
     } else if (warp == Cfg::MMA_WARP) {
         // ------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            TileScheduler<LAYOUT> sched(p);
-            TileCoord tc;
-            uint32_t stage = 0, phase = 0, acc_i = 0, committed = 0;
-            bool ok = true;
-            constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BN);
-            while (ok && sched.next(tc, false)) {
-                for (int kb = 0; kb < p.num_kb; ++kb) {
-                    const uint32_t buf = acc_i & 1, tph = (acc_i >> 1) & 1;
-                    if (!wait_bounded(smem_addr(tempty_bar + buf), tph ^ 1, tmo, abort_flag,
-                                      kRoleMma, 16 + buf, true) ||
-                        !wait_bounded(smem_addr(full_bar + stage), phase, tmo, abort_flag,
-                                      kRoleMma, stage, true)) {
+        // Uniform loop; the descriptors stay warp-uniform and one elected
+        // lane issues the MMAs and the commits.
+        TileScheduler<LAYOUT> sched(p);
+        TileCoord tc;
+        uint32_t stage = 0, phase = 0, acc_i = 0, committed = 0;
+        bool ok = true;
+        constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BN);
+        const uint64_t a_desc0 = smem_desc_k_sw128(smem_addr(a_tiles));
+        const uint64_t b_desc0 = smem_desc_k_sw128(smem_addr(b_tiles));
+        while (ok && sched.next(tc, false)) {
+            for (int kb0 = 0; kb0 < p.num_kb; kb0 += KS) {
+                if (!warp_wait_bounded(smem_addr(full_bar + stage), phase, tmo, abort_flag,
+                                       kRoleMma, stage)) {
+                    ok = false;
+                    break;
+                }
+#pragma unroll
+                for (int q = 0; q < KS; ++q) {
+                    if (kb0 + q >= p.num_kb)
+                        break;
+                    const uint32_t buf = acc_i % NBUF, tph = (acc_i / NBUF) & 1;
+                    if (!warp_wait_bounded(smem_addr(tempty_bar + buf), tph ^ 1, tmo, abort_flag,
+                                           kRoleMma, 16 + buf)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
                     const uint32_t d_tmem = tmem_base + buf * Cfg::ACC_STRIDE;
-                    const uint32_t a0 = smem_addr(a_tiles + stage * Cfg::A_BYTES);
-                    const uint32_t b0 = smem_addr(b_tiles + stage * Cfg::B_BYTES);
+                    // descriptor start address advances in 16-byte units
+                    const uint64_t ad = a_desc0 + static_cast<uint64_t>(((stage * KS + q) * Cfg::A_BYTES) >> 4);
+                    const uint64_t bd = b_desc0 + static_cast<uint64_t>(((stage * KS + q) * Cfg::B_BYTES) >> 4);
+                    if (elect_one()) {
 #pragma unroll
-                    for (int j = 0; j < kBK / 32; ++j)
-                        mma_f8f6f4(d_tmem, smem_desc_k_sw128(a0 + j * 32),
-                                   smem_desc_k_sw128(b0 + j * 32), idesc, j > 0 ? 1u : 0u);
-                    mma_commit(smem_addr(empty_bar + stage));
-                    mma_commit(smem_addr(tfull_bar + buf));
-                    ++committed;
-                    ++acc_i;
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1;
+                        for (int j = 0; j < kBK / 32; ++j)
+                            mma_f8f6f4(d_tmem, ad + 2 * j, bd + 2 * j, idesc, j > 0 ? 1u : 0u);
+                        mma_commit(smem_addr(tfull_bar + buf));
                     }
+                    __syncwarp();
+                    ++acc_i;
+                }
+                if (!ok)
+                    break;
+                if (elect_one())
+                    mma_commit(smem_addr(empty_bar + stage));
+                __syncwarp();
+                ++committed;
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
                 }
             }
-            // Drain: the last commit (to the empty barrier of the last stage
-            // used) fires once every MMA issued by this thread has finished.
-            if (committed > 0) {
-                const uint32_t i = committed - 1;
-                wait_bounded(smem_addr(empty_bar + i % STAGES), (i / STAGES) & 1, tmo, abort_flag,
-                             kRoleDrain, 32 + i % STAGES, false);
-            }
+        }
+        // Drain: the last commit (to the empty barrier of the last stage
+        // used) fires once every MMA issued by this warp has finished.
+        if (lane == 0 && committed > 0) {
+            const uint32_t i = committed - 1;
+            wait_bounded(smem_addr(empty_bar + i % STAGES), (i / STAGES) & 1, tmo, abort_flag,
+                         kRoleDrain, 32 + i % STAGES, false);
         }
         __syncwarp();
     } else {
@@ -359,10 +488,11 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES>::THREADS, 1)
         const int wg = warp / 4;
         const int quad = warp % 4;
         const int row = quad * 32 + lane;  // tile row == TMEM lane
+        const int wg_tid = threadIdx.x % 128;
         const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
         TileScheduler<LAYOUT> sched(p);
         TileCoord tc;
-        uint32_t acc_i = 0;
+        uint32_t acc_i = 0, stage = 0, phase = 0;
         bool ok = true;
         float acc[BN_WG];
 
@@ -384,94 +514,143 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES>::THREADS, 1)
                 mm = mm < 0 ? 0 : (mm > p.M ? p.M : mm);
                 row_ok = m_local < mm;
             }
-            const float *sa_ptr = p.sA +
-                                  (LAYOUT == kMasked ? static_cast<size_t>(tc.g) * p.num_kb * p.sa_ld
-                                                     : 0) +
-                                  m_local;
             const int col0 = tc.nb * BN + wg * BN_WG;  // first column of this warpgroup
+            const int nb_first = (tc.nb * BN) / 128;   // block of sb slot 0
             const int nb_lo = min(col0 / 128, p.nbn - 1);
-            const int nb_hi = min(nb_lo + 1, p.nbn - 1);
+            const int j_lo = nb_lo - nb_first;
+            const int j_hi = min(nb_lo + 1, p.nbn - 1) - nb_first;
             const int boundary = (nb_lo + 1) * 128 - col0;  // local column where sB switches
-            const float *sb_lo = p.sB + (static_cast<size_t>(tc.g) * p.nbn + nb_lo) * p.num_kb;
-            const float *sb_hi = p.sB + (static_cast<size_t>(tc.g) * p.nbn + nb_hi) * p.num_kb;
-
-            float sa_next = row_ok ? __ldg(sa_ptr) : 0.0f;
-            float sbl_next = __ldg(sb_lo);
-            float sbh_next = __ldg(sb_hi);
 #pragma unroll
             for (int i = 0; i < BN_WG; ++i)
                 acc[i] = 0.0f;
 
-            for (int kb = 0; kb < p.num_kb; ++kb) {
-                const float sa = sa_next, sbl = sbl_next, sbh = sbh_next;
-                if (kb + 1 < p.num_kb) {
-                    sa_next = row_ok ? __ldg(sa_ptr + static_cast<size_t>(kb + 1) * p.sa_ld) : 0.0f;
-                    sbl_next = __ldg(sb_lo + kb + 1);
-                    sbh_next = __ldg(sb_hi + kb + 1);
-                }
-                const float s_lo = sa * sbl;
-                const float s_hi = sa * sbh;
-                const uint32_t buf = acc_i & 1, tph = (acc_i >> 1) & 1;
-                if (!warp_wait_bounded(smem_addr(tfull_bar + buf), tph, tmo, abort_flag,
-                                       kRolePromote, 16 + buf)) {
+            for (int kb0 = 0; kb0 < p.num_kb; kb0 += KS) {
+                // the stage's scales, then hand the scale slots back
+                if (!warp_wait_bounded(smem_addr(full_bar + stage), phase, tmo, abort_flag,
+                                       kRolePromote, stage)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after_sync();
-                const uint32_t taddr = tmem_base + lane_bits + buf * Cfg::ACC_STRIDE + wg * BN_WG;
+                float s_lo[KS], s_hi[KS];
 #pragma unroll
-                for (int c = 0; c < CHUNKS; c += 2) {
-                    uint32_t r0[16], r1[16];
-                    tmem_ld_32x32b_x16(taddr + c * 16, r0);
-                    if (c + 1 < CHUNKS)
-                        tmem_ld_32x32b_x16(taddr + (c + 1) * 16, r1);
-                    tmem_ld_wait();
-                    if (c + 2 >= CHUNKS) {
-                        // every column of this buffer is in registers: free it
-                        tc_fence_before_sync();
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(smem_addr(tempty_bar + buf));
-                    }
-                    const float s0 = (c * 16 >= boundary) ? s_hi : s_lo;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        acc[c * 16 + i] = fmaf(__uint_as_float(r0[i]), s0, acc[c * 16 + i]);
-                    if (c + 1 < CHUNKS) {
-                        const float s1 = ((c + 1) * 16 >= boundary) ? s_hi : s_lo;
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            acc[(c + 1) * 16 + i] =
-                                fmaf(__uint_as_float(r1[i]), s1, acc[(c + 1) * 16 + i]);
-                    }
+                for (int q = 0; q < KS; ++q) {
+                    const float sa = sa_tiles[(stage * KS + q) * kBM + row];
+                    s_lo[q] = sa * sb_tiles[(stage * KS + q) * 4 + j_lo];
+                    s_hi[q] = sa * sb_tiles[(stage * KS + q) * 4 + j_hi];
                 }
-                ++acc_i;
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_addr(sread_bar + stage));
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+#pragma unroll
+                for (int q = 0; q < KS; ++q) {
+                    if (kb0 + q >= p.num_kb)
+                        break;
+                    const uint32_t buf = acc_i % NBUF, tph = (acc_i / NBUF) & 1;
+                    if (!warp_wait_bounded(smem_addr(tfull_bar + buf), tph, tmo, abort_flag,
+                                           kRolePromote, 16 + buf)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t taddr = tmem_base + lane_bits + buf * Cfg::ACC_STRIDE + wg * BN_WG;
+#pragma unroll
+                    for (int c0 = 0; c0 < BN_WG; c0 += RMAX) {
+                        constexpr int TAIL = BN_WG % RMAX;
+                        uint32_t r[RMAX];
+                        const bool whole = c0 + RMAX <= BN_WG;
+                        if (whole)
+                            tmem_load_cols<RMAX>(taddr + c0, r);
+                        else
+                            tmem_load_cols<TAIL>(taddr + c0, r);
+                        tmem_ld_wait();
+                        if (c0 + RMAX >= BN_WG) {
+                            // every column of this buffer is in registers: free it
+                            tc_fence_before_sync();
+                            __syncwarp();
+                            if (lane == 0)
+                                mbar_arrive(smem_addr(tempty_bar + buf));
+                        }
+#pragma unroll
+                        for (int g8 = 0; g8 < RMAX; g8 += 8) {
+                            if (whole || g8 < TAIL) {
+                                const float sc = (c0 + g8 >= boundary) ? s_hi[q] : s_lo[q];
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    acc[c0 + g8 + i] = fmaf(__uint_as_float(r[g8 + i]), sc, acc[c0 + g8 + i]);
+                            }
+                        }
+                    }
+                    ++acc_i;
+                }
+                if (!ok)
+                    break;
             }
-            if (!ok)
-                break;
 
             // ------------------------------------------------------ epilogue
-            if (row_ok) {
+            // A warpgroup stores its 128 rows with whole-tile TMA boxes when
+            // every row may be written: dense rows past M are clipped by the
+            // tensor extent, while grouped layouts must not touch rows outside
+            // the group, so a warpgroup with any such row stores row by row.
+            // A warp that gave up on a wait still joins this first barrier
+            // (voting "no"), so no warp of its warpgroup waits for it at a
+            // named barrier; it then leaves.
+            const bool tile_rows_ok = named_barrier_and(
+                1 + wg, 128, ok && (LAYOUT == kDense ? (tc.mb * kBM < p.M) : row_ok));
+            if (!ok)
+                break;
+            if (tile_rows_ok) {
+                const int grow0 = (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * kBM;
+                const uint32_t stg = smem_addr(epi_stage + wg * Cfg::EPI_WG_BYTES);
+#pragma unroll
+                for (int bx = 0; bx < Cfg::EPI_FULL_BOXES + (Cfg::EPI_REM > 0 ? 1 : 0); ++bx) {
+                    const bool full = bx < Cfg::EPI_FULL_BOXES;
+                    const int cbase = bx * 64;
+                    const int ncols = full ? 64 : Cfg::EPI_REM;
+                    if (col0 + cbase >= p.N)
+                        break;  // this box (and any after it) lies past N
+                    // the previous store from this staging buffer must have
+                    // finished reading it before it is overwritten
+                    if (wg_tid == 0)
+                        bulk_wait_group_read<0>();
+                    named_barrier_sync(1 + wg, 128);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        if (ch * 8 < ncols) {
+                            // full boxes: 128-byte rows, 16-byte chunk index
+                            // XOR (row % 8); remainder: dense rows of ncols*2
+                            const uint32_t off =
+                                full ? static_cast<uint32_t>(row * 128 + ((ch ^ (row & 7)) * 16))
+                                     : static_cast<uint32_t>(row * ncols * 2 + ch * 16);
+                            st_shared_v4(stg + off, pack_bf16x8(acc + cbase + ch * 8));
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    named_barrier_sync(1 + wg, 128);
+                    if (wg_tid == 0) {
+                        tma_store_2d(full ? static_cast<const void *>(&tmap_d64)
+                                          : static_cast<const void *>(&tmap_drem),
+                                     stg, col0 + cbase, grow0);
+                        bulk_commit_group();
+                    }
+                }
+            } else if (row_ok) {
                 const size_t grow = (LAYOUT == kMasked ? static_cast<size_t>(tc.g) * p.M : 0) +
                                     static_cast<size_t>(m_local);
                 __nv_bfloat16 *drow = p.D + grow * p.N + col0;
 #pragma unroll
-                for (int c = 0; c < BN_WG; c += 8) {
-                    if (col0 + c < p.N) {
-                        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc[c + 0], acc[c + 1]);
-                        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc[c + 2], acc[c + 3]);
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[c + 4], acc[c + 5]);
-                        __nv_bfloat162 h3 = __floats2bfloat162_rn(acc[c + 6], acc[c + 7]);
-                        uint4 v;
-                        v.x = *reinterpret_cast<uint32_t *>(&h0);
-                        v.y = *reinterpret_cast<uint32_t *>(&h1);
-                        v.z = *reinterpret_cast<uint32_t *>(&h2);
-                        v.w = *reinterpret_cast<uint32_t *>(&h3);
-                        *reinterpret_cast<uint4 *>(drow + c) = v;
-                    }
-                }
+                for (int c = 0; c < BN_WG; c += 8)
+                    if (col0 + c < p.N)
+                        *reinterpret_cast<uint4 *>(drow + c) = pack_bf16x8(acc + c);
             }
         }
+        // all output stores of this warpgroup complete before the CTA exits
+        if (wg_tid == 0)
+            bulk_wait_group<0>();
+        __syncwarp();
     }
 
     __syncthreads();
