@@ -41,7 +41,15 @@
  *    past its time limit) never trap: the kernel records a code in a device
  *    status word, leaves the affected rows untouched and returns.  Read and
  *    clear it with dg_get_device_status().
- *  - The library allocates no device memory for a GEMM call.
+ *  - Device memory: the persistent paths allocate nothing.  For dense shapes
+ *    with too few output tiles to fill the GPU (decode shapes), the library
+ *    splits each tile's K range over a cluster of 2..16 CTAs whose fp32
+ *    partial tiles meet in a library-owned workspace (tiles x splits x
+ *    BN x 128 floats; 8.6 MB for M=128, N=2112, K=7168).  It is allocated on
+ *    the first such call on a device, grown when a larger one is needed and
+ *    kept until exit -- so make that first call before any stream capture.
+ *    Calls that take this path on one device share the workspace: they must
+ *    not overlap on the GPU (issue them on one stream).
  *  - Layout constraints: K >= 128 and K % 128 == 0; N >= 16 and N % 16 == 0;
  *    A, B, D and sA 16-byte aligned; sB and the metadata 4-byte aligned.
  *  - Row-major, packed (no leading-dimension arguments).

@@ -115,6 +115,36 @@ int effective_sms(int dev)
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Per-device fp32 workspace of the K-split path, allocated on first use and
+// grown when a larger one is needed; kept until process exit.
+std::mutex g_ws_mutex;
+void *g_ws_ptr[kMaxDevices] = {};
+size_t g_ws_bytes[kMaxDevices] = {};
+
+dg_status_t split_workspace(int dev, size_t bytes, void **out)
+{
+    if (dev < 0 || dev >= kMaxDevices)
+        return DG_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    if (g_ws_bytes[dev] < bytes) {
+        if (g_ws_ptr[dev]) {
+            if (cudaFree(g_ws_ptr[dev]) != cudaSuccess)
+                return DG_ERR_CUDA;
+            g_ws_ptr[dev] = nullptr;
+            g_ws_bytes[dev] = 0;
+        }
+        void *ptr = nullptr;
+        if (cudaMalloc(&ptr, bytes) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return DG_ERR_CUDA;
+        }
+        g_ws_ptr[dev] = ptr;
+        g_ws_bytes[dev] = bytes;
+    }
+    *out = g_ws_ptr[dev];
+    return DG_OK;
+}
+
 // ---------------------------------------------------------- configurations
 
 // The tile widths compiled into the library.  Each has a pipeline depth that
@@ -122,14 +152,17 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 struct TileChoice {
     int bn;
     int stages;
-    int ks;  // 128-wide K blocks per pipeline stage
+    int ks;      // 128-wide K blocks per pipeline stage
+    int split;   // 0: persistent tiles; 1: K split over a cluster (dense only)
+    double kb_ns;  // measured time of one K block of one tile (cost model)
 };
-constexpr TileChoice kTileChoices[] = {{112, 3, 2}, {128, 5, 1}, {224, 2, 2}, {256, 3, 1}};
+constexpr TileChoice kTileChoices[] = {
+    {112, 3, 2, 0, 0.41}, {128, 5, 1, 0, 0.53}, {224, 2, 2, 0, 0.78}, {256, 3, 1, 0, 0.68},
+    {144, 3, 2, 1, 0.40},
+};
+constexpr int kNumChoices = sizeof(kTileChoices) / sizeof(kTileChoices[0]);
+constexpr int kSplitFixedNs = 1500;  // cluster reduction + pipeline fill of a split CTA
 
-// Deterministic choice, no autotuning (lqnn.cn article, section
-// "完全JIT设计"; non-power-of-two BLOCK_N to fill the SMs, section
-// "非对齐块大小"): the number of waves of tiles over the SMs times the time of
-// one tile, which grows with BN plus a fixed per-tile cost.
 // DG_FORCE_BLOCK_N=<n> pins the tile width to one of the compiled choices
 // (read once; for tuning sweeps).
 int forced_block_n()
@@ -142,23 +175,52 @@ int forced_block_n()
     return v;
 }
 
-TileChoice choose_tile(int64_t m_blocks, int N, int sms)
+struct Plan {
+    TileChoice c;
+    int ksplit;  // CTAs per cluster sharing a tile's K range (1 = none)
+};
+
+int max_active_clusters(const TileChoice &c, int S);
+
+// Deterministic choice, no autotuning (lqnn.cn article, section
+// "完全JIT设计"; non-power-of-two BLOCK_N to fill the SMs, section
+// "非对齐块大小"): waves of tiles over the SMs times the time of one tile.
+// When a problem has too few tiles to fill the GPU (decode shapes), the K
+// range of each tile may be split over a cluster of 2..16 CTAs.
+Plan choose_plan(int64_t m_blocks, int N, int num_kb, int sms, bool allow_split)
 {
-    for (const TileChoice &c : kTileChoices)
-        if (c.bn == forced_block_n())
-            return c;
-    TileChoice best = kTileChoices[0];
+    Plan best{kTileChoices[0], 1};
     double best_cost = 1e300;
     for (const TileChoice &c : kTileChoices) {
-        const int64_t n_blocks = (N + c.bn - 1) / c.bn;
-        const int64_t tiles = m_blocks * n_blocks;
-        const int64_t waves = (tiles + sms - 1) / sms;
-        // time of one tile ~ BN (MMA + promotion columns) + fixed overhead;
-        // columns beyond N in the last n-block are wasted work.
-        const double cost = static_cast<double>(waves) * (c.bn + 32);
-        if (cost < best_cost - 1e-9 || (cost < best_cost + 1e-9 && c.bn > best.bn)) {
-            best_cost = cost;
-            best = c;
+        const bool forced = forced_block_n() > 0;
+        if (forced && c.bn != forced_block_n())
+            continue;
+        const int64_t tiles = m_blocks * ((N + c.bn - 1) / c.bn);
+        if (!c.split) {
+            const int64_t waves = (tiles + sms - 1) / sms;
+            const double cost = static_cast<double>(waves) * num_kb * c.kb_ns;
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = Plan{c, 1};
+            }
+            continue;
+        }
+        if (!allow_split)
+            continue;
+        for (int S = 2; S <= 16; S *= 2) {
+            const int kbps = (num_kb + S - 1) / S;
+            if (kbps < 2)
+                break;
+            const int S_eff = (num_kb + kbps - 1) / kbps;
+            if (S_eff != S)
+                continue;
+            if (tiles > max_active_clusters(c, S))
+                continue;
+            const double cost = kbps * c.kb_ns + kSplitFixedNs * 1e-3;
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = Plan{c, S};
+            }
         }
     }
     return best;
@@ -169,11 +231,11 @@ int choose_raster(int num_mb)
     return num_mb < 16 ? (num_mb > 0 ? num_mb : 1) : 16;
 }
 
-template <int BN, int STAGES, int KS, int LAYOUT>
+template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT>
 dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
                           const GemmParams &p, int grid, cudaStream_t stream)
 {
-    using Cfg = KernelConfig<BN, STAGES, KS>;
+    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT>;
     CUtensorMap ta, tb;
     if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
         !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, BN, KS))
@@ -192,7 +254,7 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
     } else {
         tdrem = td64;
     }
-    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT>;
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT, SPLIT>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices)
@@ -201,7 +263,29 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg::SMEM_BYTES) != cudaSuccess)
             return DG_ERR_CUDA;
+        if (SPLIT && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                         cudaSuccess)
+            return DG_ERR_CUDA;
         attr_set[dev].store(true);
+    }
+    if (SPLIT) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+        cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(p.ksplit);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, ta, tb, td64, tdrem, p) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return DG_ERR_CUDA;
+        }
+        return DG_OK;
     }
     kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, td64, tdrem, p);
     if (cudaPeekAtLastError() != cudaSuccess) {
@@ -211,26 +295,94 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
     return DG_OK;
 }
 
+// Co-resident clusters of S CTAs of a split configuration (cached per
+// device).  The split kernel keeps one tile per cluster, so a plan is only
+// used when every cluster of the grid fits at once.
+template <int BN, int STAGES, int KS>
+int query_max_clusters(int S)
+{
+    using Cfg = KernelConfig<BN, STAGES, KS, true>;
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, dg::kDense, true>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(S * 16), 1, 1);
+    cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+int max_active_clusters(const TileChoice &c, int S)
+{
+    static int cache[kMaxDevices][5] = {};  // S = 2, 4, 8, 16 (index log2(S))
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices || c.bn != 144)
+        return 0;
+    int idx = 0;
+    while ((2 << idx) < S)
+        ++idx;
+    if (cache[dev][idx] == 0) {
+        const int n = query_max_clusters<144, 3, 2>(S);
+        cache[dev][idx] = n > 0 ? n : -1;
+    }
+    // The SM cap (dg_set_num_sms) bounds the clusters too.
+    const int cap = effective_sms(dev) / S;
+    const int n = cache[dev][idx];
+    return n < 0 ? 0 : (n < cap ? n : cap);
+}
+
 template <int LAYOUT>
-dg_status_t dispatch(const TileChoice &c, const void *A, uint64_t a_rows, const void *B,
+dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const void *B,
                      uint64_t b_rows, GemmParams p, int sms, cudaStream_t stream)
 {
+    const TileChoice &c = plan.c;
     p.num_nb = (p.N + c.bn - 1) / c.bn;
-    int grid = sms;
-    if (LAYOUT != dg::kMasked) {
-        const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
-        grid = static_cast<int>(tiles < sms ? tiles : sms);
+    p.ksplit = plan.ksplit;
+    p.kb_per_split = (p.num_kb + plan.ksplit - 1) / plan.ksplit;
+    const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
+    if (plan.ksplit > 1) {
+        const size_t bytes = static_cast<size_t>(tiles) * plan.ksplit * c.bn * dg::kBM * sizeof(float);
+        void *ws = nullptr;
+        const dg_status_t st = split_workspace(current_device(), bytes, &ws);
+        if (st != DG_OK)
+            return st;
+        p.ws = static_cast<float *>(ws);
     }
+    int grid = sms;
+    if (plan.ksplit > 1)
+        grid = static_cast<int>(tiles * plan.ksplit);
+    else if (LAYOUT != dg::kMasked)
+        grid = static_cast<int>(tiles < sms ? tiles : sms);
     if (grid <= 0)
         return DG_OK;
 #define DG_TILE_CASE(BN_, ST_, KS_)                                                         \
-    if (c.bn == BN_ && c.stages == ST_ && c.ks == KS_)                                       \
-        return launch_kernel<BN_, ST_, KS_, LAYOUT>(A, a_rows, B, b_rows, p, grid, stream);
+    if (c.bn == BN_ && c.stages == ST_ && c.ks == KS_ && !c.split)                           \
+        return launch_kernel<BN_, ST_, KS_, LAYOUT, false>(A, a_rows, B, b_rows, p, grid, stream);
     DG_TILE_CASE(112, 3, 2)
     DG_TILE_CASE(128, 5, 1)
     DG_TILE_CASE(224, 2, 2)
     DG_TILE_CASE(256, 3, 1)
 #undef DG_TILE_CASE
+    if constexpr (LAYOUT == dg::kDense) {
+        if (c.bn == 144 && c.stages == 3 && c.ks == 2 && c.split)
+            return launch_kernel<144, 3, 2, LAYOUT, true>(A, a_rows, B, b_rows, p, grid, stream);
+    }
     return DG_ERR_UNSUPPORTED;
 }
 
@@ -293,12 +445,12 @@ dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B, const 
     p.num_mb = (M + 127) / 128;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
-    const TileChoice c = choose_tile(p.num_mb, N, sms);
+    const Plan plan = choose_plan(p.num_mb, N, p.num_kb, sms, true);
     if (print_configs())
-        std::fprintf(stderr, "[dg] dense M=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n", M, N,
-                     K, c.bn, c.stages, c.ks, sms);
-    return dispatch<dg::kDense>(c, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), p, sms,
-                                stream);
+        std::fprintf(stderr, "[dg] dense M=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d ksplit=%d sms=%d\n",
+                     M, N, K, plan.c.bn, plan.c.stages, plan.c.ks, plan.ksplit, sms);
+    return dispatch<dg::kDense>(plan, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), p,
+                                sms, stream);
 }
 
 dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const void *B,
@@ -338,11 +490,11 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const
     p.num_mb = M_total / 128;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
-    const TileChoice c = choose_tile(p.num_mb, N, sms);
+    const Plan plan = choose_plan(p.num_mb, N, p.num_kb, sms, false);
     if (print_configs())
-        std::fprintf(stderr, "[dg] contiguous M=%d N=%d K=%d G=%d -> BM=128 BN=%d stages=%d sms=%d\n",
-                     M_total, N, K, num_groups, c.bn, c.stages, sms);
-    return dispatch<dg::kContiguous>(c, A, static_cast<uint64_t>(M_total), B,
+        std::fprintf(stderr, "[dg] contiguous M=%d N=%d K=%d G=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
+                     M_total, N, K, num_groups, plan.c.bn, plan.c.stages, plan.c.ks, sms);
+    return dispatch<dg::kContiguous>(plan, A, static_cast<uint64_t>(M_total), B,
                                      static_cast<uint64_t>(num_groups) * N, p, sms, stream);
 }
 
@@ -383,12 +535,13 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const voi
     p.raster = 1;
     p.timeout_ns = g_timeout_ns.load();
     const int em = (expected_m > 0 && expected_m < max_m) ? expected_m : max_m;
-    const TileChoice c = choose_tile(static_cast<int64_t>(num_groups) * ((em + 127) / 128), N, sms);
+    const Plan plan = choose_plan(static_cast<int64_t>(num_groups) * ((em + 127) / 128), N,
+                                  p.num_kb, sms, false);
     if (print_configs())
         std::fprintf(stderr,
-                     "[dg] masked G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=128 BN=%d stages=%d sms=%d\n",
-                     num_groups, max_m, em, N, K, c.bn, c.stages, sms);
-    return dispatch<dg::kMasked>(c, A, static_cast<uint64_t>(num_groups) * max_m, B,
+                     "[dg] masked G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
+                     num_groups, max_m, em, N, K, plan.c.bn, plan.c.stages, plan.c.ks, sms);
+    return dispatch<dg::kMasked>(plan, A, static_cast<uint64_t>(num_groups) * max_m, B,
                                  static_cast<uint64_t>(num_groups) * N, p, sms, stream);
 }
 
@@ -458,11 +611,12 @@ int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, i
     int64_t m_blocks = (M + 127) / 128;
     if (layout == 2)
         m_blocks *= groups;
-    const TileChoice c = choose_tile(m_blocks, N, sms);
+    const Plan plan = choose_plan(m_blocks, N, K / 128 > 0 ? K / 128 : 1, sms, layout == 0);
+    const TileChoice &c = plan.c;
     return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
-                         "layout=%d BM=128 BN=%d BK=128 stages=%d ks=%d sms=%d m_blocks=%lld n_blocks=%d",
-                         layout, c.bn, c.stages, c.ks, sms, static_cast<long long>(m_blocks),
-                         (N + c.bn - 1) / c.bn);
+                         "layout=%d BM=128 BN=%d BK=128 stages=%d ks=%d ksplit=%d sms=%d m_blocks=%lld n_blocks=%d",
+                         layout, c.bn, c.stages, c.ks, plan.ksplit, sms,
+                         static_cast<long long>(m_blocks), (N + c.bn - 1) / c.bn);
 }
 
 const char *dg_status_string(dg_status_t status)

@@ -87,6 +87,9 @@ struct GemmParams {
     int num_mb;               // dense/contig: ceil(M / 128)
     int num_nb;               // ceil(N / BN)
     int raster;               // m-blocks per rasterisation group (dense/contig)
+    int ksplit;               // CTAs of a cluster sharing one tile's K range (1 = no split)
+    int kb_per_split;         // K blocks per split
+    float *ws;                // K split: fp32 partials [tile][split][BN/4][128][4]
     unsigned long long timeout_ns;
 };
 
@@ -107,7 +110,22 @@ struct TileScheduler {
     int next_t;
     int cur_g = 0, cur_base = 0, cur_count = -1;
 
-    __device__ explicit TileScheduler(const GemmParams &params) : p(params), next_t(blockIdx.x) {}
+    int stride;
+
+    // With a K split, the ksplit CTAs of a cluster share one tile (and the
+    // grid holds exactly one tile per cluster).
+    __device__ explicit TileScheduler(const GemmParams &params)
+        : p(params), next_t(blockIdx.x / params.ksplit), stride(gridDim.x / params.ksplit) {}
+
+    // This CTA's K blocks: [begin, end).
+    __device__ int kb_begin() const
+    {
+        return p.ksplit > 1 ? static_cast<int>(blockIdx.x % p.ksplit) * p.kb_per_split : 0;
+    }
+    __device__ int kb_end() const
+    {
+        return p.ksplit > 1 ? min(p.num_kb, kb_begin() + p.kb_per_split) : p.num_kb;
+    }
 
     __device__ bool next(TileCoord &tc, bool report)
     {
@@ -131,7 +149,7 @@ struct TileScheduler {
                 ++cur_g;
                 cur_count = -1;
             }
-            next_t += gridDim.x;
+            next_t += stride;
             const int local = t - cur_base;
             const int mbs = cur_count / p.num_nb;
             tc.g = cur_g;
@@ -142,7 +160,7 @@ struct TileScheduler {
             const int total = p.num_mb * p.num_nb;
             while (next_t < total) {
                 const int t = next_t;
-                next_t += gridDim.x;
+                next_t += stride;
                 const int per = p.raster * p.num_nb;
                 const int grp = t / per;
                 const int within = t - grp * per;
@@ -209,11 +227,15 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
 // BN: tile width; STAGES: shared-memory ring depth; KS: 128-wide K blocks per
 // stage (one 3-D TMA box per operand carries all KS blocks -- the TMA engine
 // costs a roughly fixed time per instruction, so bigger boxes move more).
-template <int BN_, int STAGES_, int KS_>
+template <int BN_, int STAGES_, int KS_, bool SPLIT_ = false>
 struct KernelConfig {
     static constexpr int BN = BN_;
     static constexpr int STAGES = STAGES_;
     static constexpr int KS = KS_;
+    // SPLIT: the CTAs of a cluster split K; their fp32 partial tiles go
+    // through an L2-resident workspace and are summed by the cluster instead
+    // of being TMA-stored.
+    static constexpr bool SPLIT = SPLIT_;
     // Two promotion warpgroups split the tile's columns; thread t of each
     // owns tile row t.
     static constexpr int NUM_WG = 2;
@@ -245,7 +267,8 @@ struct KernelConfig {
     static constexpr int EPI_WG_BYTES = kBM * 128;  // 128 rows x 128 bytes
     static constexpr int PIPE_BYTES = STAGES * (STAGE_BYTES + SA_BYTES + SB_BYTES);
     static constexpr int EPI_OFFSET = (PIPE_BYTES + BAR_BYTES + 1023) / 1024 * 1024;
-    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + EPI_OFFSET + NUM_WG * EPI_WG_BYTES;
+    static constexpr int SMEM_BYTES =
+        1024 /*align slack*/ + EPI_OFFSET + (SPLIT ? 0 : NUM_WG * EPI_WG_BYTES);
 
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128: multiple of 16, <= 256");
     static_assert(BN_WG % 8 == 0, "promotion columns per warpgroup must be a multiple of 8");
@@ -255,6 +278,7 @@ struct KernelConfig {
     static_assert(KS >= 1 && KS <= 4, "K blocks per stage");
     static_assert(EPI_REM % 8 == 0, "remainder box must be whole 16-byte chunks");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+    static_assert(!SPLIT || BN_WG % 4 == 0, "split reduction works on float4 columns");
 };
 
 // Loads COLS (multiple of 8, may be 0) consecutive TMEM columns of this
@@ -287,14 +311,15 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float *v)
 
 // ------------------------------------------------------------------ kernel
 
-template <int BN, int STAGES, int KS, int LAYOUT>
-__global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
+template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT>
+__global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d64,
                     const __grid_constant__ CUtensorMap tmap_drem, const GemmParams p)
 {
-    using Cfg = KernelConfig<BN, STAGES, KS>;
+    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT>;
+    static_assert(!SPLIT || LAYOUT == kDense, "K split is implemented for the dense layout");
     constexpr int BN_WG = Cfg::BN_WG;
     constexpr int RMAX = Cfg::RMAX;
     constexpr int NBUF = Cfg::NBUF;
@@ -374,7 +399,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
             const int nb_first = (tc.nb * BN) / 128;
             const float *sb_src = p.sB + (static_cast<size_t>(tc.g) * p.nbn +
                                           min(nb_first + (lane < 3 ? lane : 0), p.nbn - 1)) * p.num_kb;
-            for (int kb0 = 0; kb0 < p.num_kb; kb0 += KS) {
+            const int kb_end = sched.kb_end();
+            for (int kb0 = sched.kb_begin(); kb0 < kb_end; kb0 += KS) {
                 if (!warp_wait_bounded(smem_addr(empty_bar + stage), phase ^ 1, tmo, abort_flag,
                                        kRoleProducer, stage) ||
                     !warp_wait_bounded(smem_addr(sread_bar + stage), phase ^ 1, tmo, abort_flag,
@@ -393,7 +419,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
 #pragma unroll
                 for (int q = 0; q < KS; ++q) {
                     const int kb = kb0 + q;
-                    const bool in_k = kb < p.num_kb;
+                    const bool in_k = kb < kb_end;
                     const bool sa_ok = in_k && sa_lane_ok;
                     cp_async_16(smem_addr(sa_tiles + (stage * KS + q) * kBM) + 16 * lane,
                                 sa_ok ? static_cast<const void *>(sa_base + static_cast<size_t>(kb) * p.sa_ld)
@@ -401,7 +427,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
                                 sa_ok ? 16u : 0u);
                     if (lane < 3)
                         cp_async_4(smem_addr(sb_tiles + (stage * KS + q) * 4) + 4 * lane,
-                                   sb_src + (in_k ? kb : p.num_kb - 1));
+                                   sb_src + (in_k ? kb : kb_end - 1));
                 }
                 cp_async_mbar_arrive_noinc(fb);
                 __syncwarp();
@@ -421,6 +447,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
                              kRoleDrain, i % STAGES, false);
         }
         __syncwarp();
+        if constexpr (SPLIT)
+            cluster_sync();  // first cluster barrier of the K-split reduction
     } else if (warp == Cfg::MMA_WARP) {
         // ------------------------------------------------------- MMA issuer
         // Uniform loop; the descriptors stay warp-uniform and one elected
@@ -433,7 +461,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
         const uint64_t a_desc0 = smem_desc_k_sw128(smem_addr(a_tiles));
         const uint64_t b_desc0 = smem_desc_k_sw128(smem_addr(b_tiles));
         while (ok && sched.next(tc, false)) {
-            for (int kb0 = 0; kb0 < p.num_kb; kb0 += KS) {
+            const int kb_end = sched.kb_end();
+            for (int kb0 = sched.kb_begin(); kb0 < kb_end; kb0 += KS) {
                 if (!warp_wait_bounded(smem_addr(full_bar + stage), phase, tmo, abort_flag,
                                        kRoleMma, stage)) {
                     ok = false;
@@ -441,7 +470,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
                 }
 #pragma unroll
                 for (int q = 0; q < KS; ++q) {
-                    if (kb0 + q >= p.num_kb)
+                    if (kb0 + q >= kb_end)
                         break;
                     const uint32_t buf = acc_i % NBUF, tph = (acc_i / NBUF) & 1;
                     if (!warp_wait_bounded(smem_addr(tempty_bar + buf), tph ^ 1, tmo, abort_flag,
@@ -483,6 +512,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
                          kRoleDrain, 32 + i % STAGES, false);
         }
         __syncwarp();
+        if constexpr (SPLIT)
+            cluster_sync();  // first cluster barrier of the K-split reduction
     } else {
         // ------------------------------------------------ promotion warps
         const int wg = warp / 4;
@@ -524,7 +555,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
             for (int i = 0; i < BN_WG; ++i)
                 acc[i] = 0.0f;
 
-            for (int kb0 = 0; kb0 < p.num_kb; kb0 += KS) {
+            const int kb_end = sched.kb_end();
+            for (int kb0 = sched.kb_begin(); kb0 < kb_end; kb0 += KS) {
                 // the stage's scales, then hand the scale slots back
                 if (!warp_wait_bounded(smem_addr(full_bar + stage), phase, tmo, abort_flag,
                                        kRolePromote, stage)) {
@@ -547,7 +579,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
                 }
 #pragma unroll
                 for (int q = 0; q < KS; ++q) {
-                    if (kb0 + q >= p.num_kb)
+                    if (kb0 + q >= kb_end)
                         break;
                     const uint32_t buf = acc_i % NBUF, tph = (acc_i / NBUF) & 1;
                     if (!warp_wait_bounded(smem_addr(tfull_bar + buf), tph, tmo, abort_flag,
@@ -591,6 +623,20 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
             }
 
             // ------------------------------------------------------ epilogue
+            if constexpr (SPLIT) {
+                // K split: this split's fp32 partial tile goes to the
+                // workspace as [column quad][row] float4s, so the 32 rows of
+                // a warp write 512 contiguous bytes per store.
+                if (ok) {
+                    const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
+                    float4 *dst = reinterpret_cast<float4 *>(p.ws) +
+                                  ((tile * p.ksplit + cluster_ctarank()) * (BN / 4) + wg * (BN_WG / 4)) * kBM + row;
+#pragma unroll
+                    for (int c = 0; c < BN_WG; c += 4)
+                        dst[(c / 4) * kBM] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                }
+                continue;
+            }
             // A warpgroup stores its 128 rows with whole-tile TMA boxes when
             // every row may be written: dense rows past M are clipped by the
             // tensor extent, while grouped layouts must not touch rows outside
@@ -647,6 +693,10 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
                         *reinterpret_cast<uint4 *>(drow + c) = pack_bf16x8(acc + c);
             }
         }
+        if constexpr (SPLIT) {
+            __threadfence();
+            cluster_sync();  // every split's partial tile is in the workspace
+        }
         // all output stores of this warpgroup complete before the CTA exits
         if (wg_tid == 0)
             bulk_wait_group<0>();
@@ -654,6 +704,45 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS>::THREADS, 1)
     }
 
     __syncthreads();
+    if constexpr (SPLIT) {
+        // K-split reduction: CTA `rank` owns rows [rank*128/S, (rank+1)*128/S)
+        // of the tile and sums the S partials of those rows from the
+        // workspace in split order (a fixed order, so results do not depend
+        // on timing), then rounds to bf16.
+        const int S = p.ksplit;
+        const uint32_t rank = cluster_ctarank();
+        TileScheduler<LAYOUT> sched(p);
+        TileCoord tc;
+        if (sched.next(tc, false)) {
+            const int rows_per = kBM / S;
+            constexpr int C4 = BN / 4;
+            const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
+            const float4 *src0 = reinterpret_cast<const float4 *>(p.ws) + tile * S * C4 * kBM;
+            for (int it = threadIdx.x; it < rows_per * C4; it += Cfg::THREADS) {
+                const int lr = it % rows_per;  // rows fastest: contiguous reads
+                const int c4 = it / rows_per;
+                const int r = static_cast<int>(rank) * rows_per + lr;
+                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int src = 0; src < S; ++src) {
+                    const float4 v = __ldcg(src0 + (static_cast<size_t>(src) * C4 + c4) * kBM + r);
+                    sum.x += v.x;
+                    sum.y += v.y;
+                    sum.z += v.z;
+                    sum.w += v.w;
+                }
+                const int grow = tc.mb * kBM + r;
+                const int gcol = tc.nb * BN + c4 * 4;
+                if (grow < p.M && gcol < p.N) {
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
+                    uint2 u;
+                    u.x = *reinterpret_cast<uint32_t *>(&h0);
+                    u.y = *reinterpret_cast<uint32_t *>(&h1);
+                    *reinterpret_cast<uint2 *>(p.D + static_cast<size_t>(grow) * p.N + gcol) = u;
+                }
+            }
+        }
+    }
     if (warp == Cfg::MMA_WARP) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);

@@ -47,6 +47,11 @@ def _run_dense(dg, p):
     (256, 1024, 1024),
     (300, 2112, 640),
     (513, 7168, 256),     # wide N: 224/256-column tiles, ragged M tail
+    # decode shapes: too few tiles to fill the GPU, so the K range of each
+    # tile is split over a cluster and reduced through distributed shared memory
+    (128, 1024, 4096),
+    (64, 2112, 7168),
+    (100, 4096, 3200),    # 25 K blocks: uneven split
 ])
 def test_dense_matches_oracle(dg, oracle_mod, M, N, K):
     p = gi.dense_problem(M, N, K, seed_a=1000 + M, seed_b=2000 + N)
@@ -234,8 +239,10 @@ def test_num_sms_cap_gives_same_result(dg):
     assert np.array_equal(full, capped)
 
 
-def test_repeated_calls_deterministic(dg):
-    p = gi.dense_problem(384, 2112, 1024, seed_a=51, seed_b=52)
+@pytest.mark.parametrize("M,N,K", [(384, 2112, 1024), (128, 2112, 7168)])
+def test_repeated_calls_deterministic(dg, M, N, K):
+    # the second shape takes the K-split path: its reduction order is fixed
+    p = gi.dense_problem(M, N, K, seed_a=51, seed_b=52)
     a = _run_dense(dg, p)
     b = _run_dense(dg, p)
     assert np.array_equal(a, b)
