@@ -71,7 +71,9 @@ typedef enum {
     DG_ERR_ALIGNMENT = 3,      /* pointer not aligned as required            */
     DG_ERR_CUDA = 4,           /* a CUDA runtime or driver call failed       */
     DG_ERR_TIMEOUT = 5,        /* device: a pipeline wait ran out of time    */
-    DG_ERR_BAD_GROUP_DATA = 6  /* device: m_indices / masked_m out of range  */
+    DG_ERR_BAD_GROUP_DATA = 6, /* device: m_indices / masked_m out of range  */
+    DG_ERR_WORKSPACE_LIMIT = 7 /* problem too large for the fixed scratch of
+                                  dg_fp8_gemm_nt_noalloc                    */
 } dg_status_t;
 
 /*
@@ -130,6 +132,35 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA,
                                        const int32_t *masked_m, int num_groups,
                                        int max_m, int N, int K, int expected_m,
                                        cudaStream_t stream);
+
+/*
+ * Dense NT GEMM that allocates no device memory (same arguments, layouts
+ * and result as dg_fp8_gemm_nt).  The pages describe no such call; it exists
+ * for callers that cannot call cudaMalloc while they run: code being
+ * captured into a CUDA graph (allocation is not allowed during capture),
+ * code whose framework owns all device memory through its own caching pool,
+ * and latency-critical loops where the device-wide synchronisation that
+ * cudaMalloc/cudaFree may imply is not acceptable.
+ *
+ * It runs the K-split kernel (128 x 144 tiles, each tile's K range split
+ * over a cluster of S = 1..16 CTAs) with the fp32 partials in a fixed
+ * 32 MiB array compiled into the library, which every GPU that loads the
+ * library holds until the process exits.  The partials of one call take
+ * ceil(M/128) * ceil(N/144) * S * 73,728 bytes; S is lowered until they fit,
+ * and a problem that does not fit even with S = 1 is rejected with
+ * DG_ERR_WORKSPACE_LIMIT before anything is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call uses the same array, and each call writes every part of it
+ *    that it later reads, so nothing has to start at zero.  Two calls that
+ *    overlap on the GPU (different streams, or a graph that runs them
+ *    concurrently) race on the array: serialise them.
+ *  - No cudaMalloc, cudaFree or other allocating routine is called.
+ */
+dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, const void *B,
+                                   const float *sB, void *D, int M, int N, int K,
+                                   cudaStream_t stream);
 
 /* Row alignment of each group's segment in the contiguous layout (128). */
 int dg_get_mk_alignment_for_contiguous_layout(void);

@@ -30,6 +30,7 @@ DG_OK = 0
 STATUS_NAMES = {
     0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_UNSUPPORTED", 3: "DG_ERR_ALIGNMENT",
     4: "DG_ERR_CUDA", 5: "DG_ERR_TIMEOUT", 6: "DG_ERR_BAD_GROUP_DATA",
+    7: "DG_ERR_WORKSPACE_LIMIT",
 }
 LAYOUT_DENSE, LAYOUT_CONTIGUOUS, LAYOUT_MASKED = 0, 1, 2
 
@@ -38,6 +39,7 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SIGNATURES = {
     "dg_fp8_gemm_nt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_grouped_gemm_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_fp8_grouped_gemm_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "dg_get_mk_alignment_for_contiguous_layout": (_I, []),
@@ -158,6 +160,39 @@ def dg_describe_config(layout: int, M: int, N: int, K: int, groups: int = 1) -> 
 
 def dg_status_string(status: int) -> str:
     return load_library().dg_status_string(status).decode()
+
+
+def _dense_args(A, sA, B, sB, D):
+    pa = _dev(A, "A", _FP8, 2)
+    M, K = A.shape
+    N = B.shape[0] if B.dim() == 2 else -1
+    pb = _dev(B, "B", _FP8, 2)
+    if B.shape[1] != K:
+        raise ValueError("B must be [N, K]")
+    psa = _dev(sA, "sA", _F32, 2)
+    if tuple(sA.shape) != (K // 128, get_tma_aligned_size(M, 4)):
+        raise ValueError(f"sA must be [K/128, M_pad] = {(K // 128, get_tma_aligned_size(M, 4))}")
+    psb = _dev(sB, "sB", _F32, 2)
+    if tuple(sB.shape) != ((N + 127) // 128, K // 128):
+        raise ValueError("sB must be [ceil(N/128), K/128]")
+    pd = _dev(D, "D", _BF16, 2)
+    if tuple(D.shape) != (M, N):
+        raise ValueError("D must be [M, N]")
+    return pa, psa, pb, psb, pd, M, N, K
+
+
+def dg_fp8_gemm_nt_noalloc(A, sA, B, sB, D, stream=None) -> None:
+    """Dense GEMM that allocates no device memory (for callers that cannot
+    call cudaMalloc while they run: code under CUDA-graph capture, code whose
+    framework owns all device memory in its own pool, latency-critical
+    loops).  Its K-split partials live in a fixed 32 MiB array inside the
+    library; problems that need more raise DGError(DG_ERR_WORKSPACE_LIMIT).
+    Calls share that array, so calls that could overlap on the GPU must be
+    serialised."""
+    pa, psa, pb, psb, pd, M, N, K = _dense_args(A, sA, B, sB, D)
+    st = load_library().dg_fp8_gemm_nt_noalloc(pa, psa, pb, psb, pd, M, N, K,
+                                               _stream_handle(stream, A.device))
+    _check("dg_fp8_gemm_nt_noalloc", st)
 
 
 def dg_fp8_gemm_nt(A, sA, B, sB, D, stream=None) -> None:

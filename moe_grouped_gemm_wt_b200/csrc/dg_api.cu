@@ -629,8 +629,122 @@ const char *dg_status_string(dg_status_t status)
     case DG_ERR_CUDA: return "DG_ERR_CUDA";
     case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT";
     case DG_ERR_BAD_GROUP_DATA: return "DG_ERR_BAD_GROUP_DATA";
+    case DG_ERR_WORKSPACE_LIMIT: return "DG_ERR_WORKSPACE_LIMIT";
     }
     return "DG_ERR_UNKNOWN";
 }
 
 }  // extern "C"
+
+// ====================================================== no-allocation variant
+//
+// dg_fp8_gemm_nt_noalloc: the dense GEMM through the K-split kernel, with the
+// split partials in a fixed array compiled into this library instead of a
+// workspace obtained with cudaMalloc.  For callers that must not allocate
+// device memory while they run: code being captured into a CUDA graph
+// (allocation is not allowed during capture), code whose framework keeps
+// all device memory in its own caching pool (an allocation behind its back
+// can fail or fragment that pool), and latency-critical loops where the
+// device-wide synchronisation that cudaMalloc/cudaFree may imply is not
+// acceptable.
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+}
+
+// The fixed scratch.  Every GPU that loads this library holds it until the
+// process exits.  Host code must not use this name as a device address (on
+// the host it is only a stand-in symbol); the set-up below asks the runtime
+// for the real address on each device.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+namespace {
+std::mutex g_noalloc_mutex;
+float *g_noalloc_addr[kMaxDevices] = {};
+
+// Once per device, with that device current: the device address of the
+// fixed scratch.
+dg_status_t noalloc_scratch_address(float **out)
+{
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices)
+        return DG_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+            (void)cudaGetLastError();
+            return DG_ERR_CUDA;
+        }
+        g_noalloc_addr[dev] = static_cast<float *>(ptr);
+    }
+    *out = g_noalloc_addr[dev];
+    return DG_OK;
+}
+}  // namespace
+
+extern "C" dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, const void *B,
+                                               const float *sB, void *D, int M, int N, int K,
+                                               cudaStream_t stream)
+{
+    if (M < 0)
+        return DG_ERR_INVALID_ARG;
+    dg_status_t st = check_common(A, sA, B, sB, D, N, K);
+    if (st != DG_OK)
+        return st;
+    if (M == 0)
+        return DG_OK;
+    const int dev = current_device();
+    const int sms = effective_sms(dev);
+    if (sms <= 0)
+        return DG_ERR_CUDA;
+
+    // The K-split kernel's tile (BN = 144).  The split count is the one the
+    // planner would use for this shape when it splits, else the largest
+    // power of two up to 16 that leaves every split at least two K blocks;
+    // it is halved until the partials fit the fixed scratch.
+    constexpr int kBN = 144;
+    GemmParams p{};
+    p.sA = sA;
+    p.sB = sB;
+    p.D = static_cast<__nv_bfloat16 *>(D);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = 1;
+    p.sa_ld = dg_get_tma_aligned_size(M, 4);
+    p.num_kb = K / 128;
+    p.nbn = (N + 127) / 128;
+    p.num_mb = (M + 127) / 128;
+    p.num_nb = (N + kBN - 1) / kBN;
+    p.raster = choose_raster(p.num_mb);
+    p.timeout_ns = g_timeout_ns.load();
+    const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
+    const Plan plan = choose_plan(p.num_mb, N, p.num_kb, sms, true);
+    int S = 1;
+    if (plan.c.split && plan.c.bn == kBN) {
+        S = plan.ksplit;
+    } else {
+        for (int cand = 16; cand >= 2; cand /= 2)
+            if ((p.num_kb + cand - 1) / cand >= 2) {
+                S = cand;
+                break;
+            }
+    }
+    const size_t per_split = static_cast<size_t>(tiles) * kBN * dg::kBM * sizeof(float);
+    while (S > 1 && per_split * S > kNoAllocScratchBytes)
+        S /= 2;
+    if (per_split * S > kNoAllocScratchBytes)
+        return DG_ERR_WORKSPACE_LIMIT;
+    p.ksplit = S;
+    p.kb_per_split = (p.num_kb + S - 1) / S;
+    st = noalloc_scratch_address(&p.ws);
+    if (st != DG_OK)
+        return st;
+    if (print_configs())
+        std::fprintf(stderr, "[dg] dense (no-alloc) M=%d N=%d K=%d -> BN=%d ksplit=%d scratch=%zu B\n",
+                     M, N, K, kBN, S, per_split * S);
+    return launch_kernel<kBN, 3, 2, dg::kDense, true>(A, static_cast<uint64_t>(M), B,
+                                                      static_cast<uint64_t>(N), p,
+                                                      static_cast<int>(tiles * S), stream);
+}

@@ -1,0 +1,85 @@
+"""The dense GEMM entry point that allocates no device memory.
+
+Some callers cannot let a library call cudaMalloc while they run: code being
+captured into a CUDA graph (allocation is not allowed during capture), code
+whose framework owns all device memory in its own caching pool, and
+latency-critical loops that cannot afford the synchronisation an allocation
+may bring.  dg_fp8_gemm_nt_noalloc serves them by keeping its K-split
+partials in a fixed array inside the library.  This file checks, through the
+C ABI, that it gives the same results as dg_fp8_gemm_nt (within the parity
+tolerance of the other tests) on two calls in a row -- the second call finds
+the first call's partials still in the shared array -- and that it frees or
+allocates nothing while it runs.
+
+It sits in a file pytest collects last, so a run that stops at the first
+failure has already run every other test; it also passes alone in a fresh
+process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import dg_inputs as gi
+from parity import assert_close, bits, dev_dense
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dg():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from moe_grouped_gemm_wt_b200 import build as b
+    b.build()
+    import moe_grouped_gemm_wt_b200 as m
+    m.load_library()
+    m.dg_set_num_sms(0)
+    assert m.dg_get_device_status() == 0
+    return m
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (128, 2112, 7168),   # the decode benchmark shape
+    (64, 1024, 2048),
+    (300, 2112, 1152),   # three row blocks, 9 K blocks (uneven split)
+])
+def test_noalloc_matches_default_entry_point_twice(dg, M, N, K):
+    p = gi.dense_problem(M, N, K, seed_a=300 + M, seed_b=400 + N)
+    A, sA, B, sB, D_ref = dev_dense(p)
+    dg.dg_fp8_gemm_nt(A, sA, B, sB, D_ref)
+    assert dg.dg_get_device_status() == 0
+    ref = bits(D_ref)
+
+    outs = [torch.empty_like(D_ref) for _ in range(2)]
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    for out in outs:
+        dg.dg_fp8_gemm_nt_noalloc(A, sA, B, sB, out)
+    assert dg.dg_get_device_status() == 0
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before, "the no-allocation entry point changed free device memory"
+
+    for i, out in enumerate(outs):
+        assert_close(bits(out), ref, f"no-alloc call {i + 1} vs dg_fp8_gemm_nt, {M}x{N}x{K}")
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch(dg):
+    # 4096 x 7168 needs 32 x 50 tiles x 73,728 bytes = 118 MB of partials even
+    # unsplit: more than the fixed 32 MiB, so nothing is launched.
+    lib = dg.load_library()
+    M, N, K = 4096, 7168, 256
+    dev = torch.device("cuda")
+    A = torch.zeros((M, K), dtype=torch.uint8, device=dev)
+    B = torch.zeros((N, K), dtype=torch.uint8, device=dev)
+    sA = torch.zeros((K // 128, M), dtype=torch.float32, device=dev)
+    sB = torch.zeros(((N + 127) // 128, K // 128), dtype=torch.float32, device=dev)
+    D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    st = lib.dg_fp8_gemm_nt_noalloc(A.data_ptr(), sA.data_ptr(), B.data_ptr(), sB.data_ptr(),
+                                    D.data_ptr(), M, N, K, None)
+    assert st == 7 and lib.dg_status_string(st) == b"DG_ERR_WORKSPACE_LIMIT"
+    with pytest.raises(dg.DGError):
+        dg.dg_fp8_gemm_nt_noalloc(A, sA, B, sB, D)
+    assert dg.dg_get_device_status() == 0
