@@ -205,6 +205,22 @@ def call(dg, p, d, stream=None):
                                       expected_m=int(np.mean(p["masked_m"])), stream=stream)
 
 
+def workload_label(p, name):
+    if p["kind"] == "dense":
+        return f"{name} M={p['M']} N={p['N']} K={p['K']}"
+    if p["kind"] == "contiguous":
+        return f"{name} G={p['G']} M_total={p['M']} N={p['N']} K={p['K']}"
+    return f"{name} G={p['G']} max_m={p['max_m']} N={p['N']} K={p['K']} sum_masked_m={int(p['masked_m'].sum())}"
+
+
+def tile_label(dg, p):
+    if p["kind"] == "dense":
+        return dg.dg_describe_config(0, p["M"], p["N"], p["K"], 1)
+    if p["kind"] == "contiguous":
+        return dg.dg_describe_config(1, p["M"], p["N"], p["K"], p["G"])
+    return dg.dg_describe_config(2, int(np.mean(p["masked_m"])), p["N"], p["K"], p["G"])
+
+
 def time_kernel(torch, dg, p, d, steps, warmup, flush):
     """Per-launch CUDA-event times (ms) with an L2 flush before each launch."""
     stream = torch.cuda.current_stream()
@@ -332,7 +348,7 @@ def run_ours(args):
     pk = peaks()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
-    p = gi.make_workload(HEADLINE)
+    p = gi.make_workload(args.workload)
     d = to_device(p, torch, dev)
     flop, byts, _ = workload_cost(p)
 
@@ -354,8 +370,8 @@ def run_ours(args):
     shapes = {}
     if not args.no_shapes:
         for name in gi.WORKLOADS:
-            q = p if name == HEADLINE else gi.make_workload(name)
-            dq = d if name == HEADLINE else to_device(q, torch, dev)
+            q = p if name == args.workload else gi.make_workload(name)
+            dq = d if name == args.workload else to_device(q, torch, dev)
             tq = time_kernel(torch, dg, q, dq, max(10, min(args.steps, 30)), 3, flush)
             mq = statistics.median(tq)
             fq, bq, rows = workload_cost(q)
@@ -366,7 +382,7 @@ def run_ours(args):
                 "frac_of_roofline": t_roof / (mq * 1e-3),
                 "valid_rows": rows,
             }
-            if name != HEADLINE:
+            if name != args.workload:
                 del dq
                 torch.cuda.empty_cache()
     clocks = sampler.stop()
@@ -383,14 +399,14 @@ def run_ours(args):
         achieved = flop / (ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp8_peak}
-    roof["traffic"] = ncu_traffic(HEADLINE)
+    roof["traffic"] = ncu_traffic(args.workload)
     roof["peak_source"] = pk["source"] + (" (fp8 = 2 x measured bf16)" if bound == "tensor" else "")
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and p["kind"] == "dense":
         rate, cores, npass, dt = cpu_oracle_rate(p, args.cpu_budget)
         cpu = {"value": rate, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-               "sample": f"{npass} whole passes of the 128x2112x7168 problem in {dt:.1f} s"}
+               "sample": f"{npass} whole passes of the {p['M']}x{p['N']}x{p['K']} problem in {dt:.1f} s"}
 
     if world > 1:
         dist.barrier()
@@ -403,10 +419,10 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3 (fp32 promotion, bf16 out)",
         "data": "synthetic (seeded N(0,1) quantised to e4m3 with 1x128 / 128x128 fp32 scales)",
-        "config": {"workload": "dense_decode M=128 N=2112 K=7168",
+        "config": {"workload": workload_label(p, args.workload),
                    "l2": "flushed before every timed launch (512 MiB write)",
                    "parallelism": f"replicas x{world}",
-                   "tile": dg.dg_describe_config(0, p["M"], p["N"], p["K"], 1)},
+                   "tile": tile_label(dg, p)},
         "roofline": roof,
         "frac_of_roofline": t_roof / (ms * 1e-3),
         "cpu_baseline": cpu,
@@ -429,6 +445,8 @@ def main():
     ap.add_argument("--no-shapes", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--workload", choices=sorted(gi.WORKLOADS), default=HEADLINE,
+                    help="workload timed as the step (default: the decode-shaped dense GEMM)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
