@@ -205,6 +205,21 @@ def call(dg, p, d, stream=None):
                                       expected_m=int(np.mean(p["masked_m"])), stream=stream)
 
 
+def reduce_max_ms(ms, dist, device, world):
+    """Max over ranks of a per-rank time (ms); every rank gets the result."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(flop_per_rank, world, ms):
+    """Whole-job throughput (TFLOPS): every rank's work over the slowest rank's time."""
+    return flop_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def workload_label(p, name):
     if p["kind"] == "dense":
         return f"{name} M={p['M']} N={p['N']} K={p['K']}"
@@ -359,11 +374,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     times = time_kernel(torch, dg, p, d, args.steps, max(args.warmup, 3), flush)
     torch.cuda.synchronize()
-    ms = sum(times) / len(times)
+    ms = reduce_max_ms(sum(times) / len(times), dist, dev, world)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
 
     # per-shape sweep (every rank runs it; rank 0 reports)
@@ -389,7 +401,7 @@ def run_ours(args):
 
     e2e_ms, h2d, d2h = time_e2e(torch, dg, p, max(10, min(args.steps, 50)), 3, dev)
 
-    value = flop * world / (ms * 1e-3) / 1e12
+    value = whole_job_value(flop, world, ms)
     bound, t_roof, fp8_peak = roofline(flop, byts, pk)
     if bound == "hbm":
         achieved = byts / (ms * 1e-3) / 1e9

@@ -183,6 +183,14 @@ int dg_get_num_sms(void);
  * default. */
 dg_status_t dg_set_wait_timeout_ns(uint64_t ns);
 
+/* Test hook for the bounded-wait path (0 = off, the default).  While on,
+ * the producer warp of CTA 0 of every GEMM launch issues no loads, so that
+ * CTA's pipeline waits never complete: they run out after the limit of
+ * dg_set_wait_timeout_ns, the kernel records DG_ERR_TIMEOUT and returns with
+ * its copies drained and TMEM freed, and the results are garbage.  Nothing
+ * faults or hangs; turn it off again before real work. */
+dg_status_t dg_set_stall_injection(int enable);
+
 /* Synchronises `stream`, then returns the device status word of the current
  * device (DG_OK if no kernel reported a problem) and clears it.  The word
  * also holds details; see dg_get_device_status_detail. */

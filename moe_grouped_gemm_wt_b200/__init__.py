@@ -47,6 +47,7 @@ _SIGNATURES = {
     "dg_set_num_sms": (_I, [_I]),
     "dg_get_num_sms": (_I, []),
     "dg_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
+    "dg_set_stall_injection": (_I, [_I]),
     "dg_get_device_status": (_I, [_P]),
     "dg_get_device_status_detail": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "dg_describe_config": (_I, [_I, _I, _I, _I, _I, ctypes.c_char_p, _I]),
@@ -137,6 +138,11 @@ def dg_get_num_sms() -> int:
 
 def dg_set_wait_timeout_ns(ns: int) -> None:
     _check("dg_set_wait_timeout_ns", load_library().dg_set_wait_timeout_ns(ns))
+
+
+def dg_set_stall_injection(enable: bool) -> None:
+    """Test hook: makes CTA 0 of every launch stall so its waits run out."""
+    _check("dg_set_stall_injection", load_library().dg_set_stall_injection(1 if enable else 0))
 
 
 def dg_get_device_status(stream=None) -> int:

@@ -23,6 +23,7 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 
 std::atomic<int> g_num_sms_cap{0};
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<int> g_stall_injection{0};
 int g_sm_count[kMaxDevices] = {0};
 
 // ------------------------------------------------------------ driver entry
@@ -445,6 +446,7 @@ dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B, const 
     p.num_mb = (M + 127) / 128;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
+    p.stall_injection = g_stall_injection.load();
     const Plan plan = choose_plan(p.num_mb, N, p.num_kb, sms, true);
     if (print_configs())
         std::fprintf(stderr, "[dg] dense M=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d ksplit=%d sms=%d\n",
@@ -490,6 +492,7 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const
     p.num_mb = M_total / 128;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
+    p.stall_injection = g_stall_injection.load();
     const Plan plan = choose_plan(p.num_mb, N, p.num_kb, sms, false);
     if (print_configs())
         std::fprintf(stderr, "[dg] contiguous M=%d N=%d K=%d G=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
@@ -534,6 +537,7 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const voi
     p.num_mb = (max_m + 127) / 128;
     p.raster = 1;
     p.timeout_ns = g_timeout_ns.load();
+    p.stall_injection = g_stall_injection.load();
     const int em = (expected_m > 0 && expected_m < max_m) ? expected_m : max_m;
     const Plan plan = choose_plan(static_cast<int64_t>(num_groups) * ((em + 127) / 128), N,
                                   p.num_kb, sms, false);
@@ -569,6 +573,12 @@ int dg_get_num_sms(void) { return effective_sms(current_device()); }
 dg_status_t dg_set_wait_timeout_ns(uint64_t ns)
 {
     g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
+    return DG_OK;
+}
+
+dg_status_t dg_set_stall_injection(int enable)
+{
+    g_stall_injection.store(enable ? 1 : 0);
     return DG_OK;
 }
 
@@ -719,6 +729,7 @@ extern "C" dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, co
     p.num_nb = (N + kBN - 1) / kBN;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
+    p.stall_injection = g_stall_injection.load();
     const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
     const Plan plan = choose_plan(p.num_mb, N, p.num_kb, sms, true);
     int S = 1;

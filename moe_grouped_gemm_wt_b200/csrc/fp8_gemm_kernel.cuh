@@ -90,6 +90,7 @@ struct GemmParams {
     int ksplit;               // CTAs of a cluster sharing one tile's K range (1 = no split)
     int kb_per_split;         // K blocks per split
     float *ws;                // K split: fp32 partials [tile][split][BN/4][128][4]
+    int stall_injection;      // test hook: CTA 0's producer issues nothing
     unsigned long long timeout_ns;
 };
 
@@ -374,6 +375,9 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    // Waits for this CTA's own copies and MMAs in flight before it exits use
+    // at least a second, however short the pipeline limit is set.
+    const uint64_t drain_tmo = tmo > 1000000000ull ? tmo : 1000000000ull;
 
     if (warp == Cfg::PRODUCER_WARP) {
         // ------------------------------------------------------ TMA producer
@@ -385,7 +389,9 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
         TileCoord tc;
         uint32_t stage = 0, phase = 0;
         uint32_t issued = 0;
-        bool ok = true;
+        // Test hook (dg_set_stall_injection): CTA 0 never fills a stage, so
+        // its consumers' waits run out and report DG_ERR_TIMEOUT.
+        bool ok = !(p.stall_injection && blockIdx.x == 0);
         while (ok && sched.next(tc, lane == 0)) {
             const int a_row = (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * kBM;
             const int b_row = tc.g * p.N + tc.nb * BN;
@@ -443,8 +449,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
         if (lane == 0) {
             const uint32_t first = issued > STAGES ? issued - STAGES : 0;
             for (uint32_t i = first; i < issued; ++i)
-                wait_bounded(smem_addr(full_bar + i % STAGES), (i / STAGES) & 1, tmo, abort_flag,
-                             kRoleDrain, i % STAGES, false);
+                wait_bounded(smem_addr(full_bar + i % STAGES), (i / STAGES) & 1, drain_tmo,
+                             abort_flag, kRoleDrain, i % STAGES, false);
         }
         __syncwarp();
         if constexpr (SPLIT)
@@ -455,7 +461,10 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
         // lane issues the MMAs and the commits.
         TileScheduler<LAYOUT> sched(p);
         TileCoord tc;
-        uint32_t stage = 0, phase = 0, acc_i = 0, committed = 0;
+        uint32_t stage = 0, phase = 0, acc_i = 0;
+        // the most recent commit (barrier, phase parity): it fires once
+        // every MMA issued before it has completed
+        uint32_t last_bar = 0, last_parity = 0;
         bool ok = true;
         constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BN);
         const uint64_t a_desc0 = smem_desc_k_sw128(smem_addr(a_tiles));
@@ -490,6 +499,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                         mma_commit(smem_addr(tfull_bar + buf));
                     }
                     __syncwarp();
+                    last_bar = smem_addr(tfull_bar + buf);
+                    last_parity = tph;
                     ++acc_i;
                 }
                 if (!ok)
@@ -497,20 +508,18 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                 if (elect_one())
                     mma_commit(smem_addr(empty_bar + stage));
                 __syncwarp();
-                ++committed;
+                last_bar = smem_addr(empty_bar + stage);
+                last_parity = phase;
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
         }
-        // Drain: the last commit (to the empty barrier of the last stage
-        // used) fires once every MMA issued by this warp has finished.
-        if (lane == 0 && committed > 0) {
-            const uint32_t i = committed - 1;
-            wait_bounded(smem_addr(empty_bar + i % STAGES), (i / STAGES) & 1, tmo, abort_flag,
-                         kRoleDrain, 32 + i % STAGES, false);
-        }
+        // Drain: every MMA issued by this warp has finished once its most
+        // recent commit has fired.
+        if (lane == 0 && last_bar != 0)
+            wait_bounded(last_bar, last_parity, drain_tmo, abort_flag, kRoleDrain, 32, false);
         __syncwarp();
         if constexpr (SPLIT)
             cluster_sync();  // first cluster barrier of the K-split reduction
@@ -641,13 +650,16 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
             // every row may be written: dense rows past M are clipped by the
             // tensor extent, while grouped layouts must not touch rows outside
             // the group, so a warpgroup with any such row stores row by row.
-            // A warp that gave up on a wait still joins this first barrier
-            // (voting "no"), so no warp of its warpgroup waits for it at a
-            // named barrier; it then leaves.
-            const bool tile_rows_ok = named_barrier_and(
-                1 + wg, 128, ok && (LAYOUT == kDense ? (tc.mb * kBM < p.M) : row_ok));
-            if (!ok)
+            // A warp that gave up on a wait still joins the first barrier
+            // below; if any warp of the warpgroup gave up, the whole
+            // warpgroup leaves together, so no warp can be left waiting at
+            // a later named barrier for warps that are gone.
+            if (!named_barrier_and(1 + wg, 128, ok)) {
+                ok = false;
                 break;
+            }
+            const bool tile_rows_ok = named_barrier_and(
+                1 + wg, 128, LAYOUT == kDense ? (tc.mb * kBM < p.M) : row_ok);
             if (tile_rows_ok) {
                 const int grow0 = (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * kBM;
                 const uint32_t stg = smem_addr(epi_stage + wg * Cfg::EPI_WG_BYTES);

@@ -1,0 +1,105 @@
+"""Do the oracle's pins catch plausible mistakes?
+
+Each case plants one mistake in a temporary copy of oracle/dg_oracle.c -- a
+wrong weight-block index, a transposed operand stride, a dropped K block, a
+lost accumulation, an exponent bias off by one, truncation instead of
+round-to-nearest-even -- builds it with gcc, and checks that at least one of
+the independent pins (torch's casts, float64 matmul of the dequantised
+inputs) rejects it.  The committed oracle itself is never modified."""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import dg_inputs as gi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "dg_oracle.c")
+
+MUTATIONS = {
+    "weight-block index n%128 instead of n/128": (
+        "sB + (int64_t)(n / DGO_BLOCK) * nkb, K);\n            if (D64)\n                D64[(int64_t)m * N + n] = v;",
+        "sB + (int64_t)(n % DGO_BLOCK) * nkb, K);\n            if (D64)\n                D64[(int64_t)m * N + n] = v;"),
+    "B row stride 1 instead of K (transposed operand)": (
+        "                                   B + (int64_t)n * K,\n                                   sB + (int64_t)(n / DGO_BLOCK) * nkb, K);\n            if (D64)\n                D64[(int64_t)m * N + n] = v;",
+        "                                   B + (int64_t)n,\n                                   sB + (int64_t)(n / DGO_BLOCK) * nkb, K);\n            if (D64)\n                D64[(int64_t)m * N + n] = v;"),
+    "first K block dropped": (
+        "    for (int kb = 0; kb < nkb; ++kb) {\n        double partial = 0.0;\n        for (int k = kb * DGO_BLOCK; k < (kb + 1) * DGO_BLOCK; ++k)\n            partial += g_lut[a_row[k]] * g_lut[b_row[k]];\n        double scale",
+        "    for (int kb = 1; kb < nkb; ++kb) {\n        double partial = 0.0;\n        for (int k = kb * DGO_BLOCK; k < (kb + 1) * DGO_BLOCK; ++k)\n            partial += g_lut[a_row[k]] * g_lut[b_row[k]];\n        double scale"),
+    "accumulation lost (acc = instead of acc +=)": (
+        "        acc += scale * partial;",
+        "        acc = scale * partial;"),
+    "e4m3 exponent bias off by one": (
+        "v = ldexp((double)(8 + m), e - 10);",
+        "v = ldexp((double)(8 + m), e - 9);"),
+    "bf16 truncation instead of round-to-nearest-even": (
+        "double nq = nearbyint(r);",
+        "double nq = floor(r);"),
+}
+
+
+def _build_variant(tmp_path, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation anchor must match the oracle source exactly once"
+    mutated = tmp_path / "dg_oracle_mut.c"
+    mutated.write_text(src.replace(old, new))
+    lib_path = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                           "-o", str(lib_path), str(mutated), "-lm"])
+    lib = ctypes.CDLL(str(lib_path))
+    P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    lib.dgo_gemm_nt.argtypes = [P, P, P, P, I, I, I, P, P]
+    lib.dgo_gemm_nt.restype = I
+    lib.dgo_decode_e4m3.argtypes = [P, P, I64]
+    lib.dgo_bf16_round.argtypes = [P, P, I64]
+    return lib
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _pins_pass(lib) -> bool:
+    """The independent pins of test_oracle_pins, run against `lib`."""
+    # decode: all 256 codes vs torch
+    codes = np.arange(256, dtype=np.uint8)
+    dec = np.empty(256, np.float64)
+    lib.dgo_decode_e4m3(_ptr(codes), _ptr(dec), 256)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    fin = ~np.isnan(ref)
+    if not np.array_equal(dec[fin], ref[fin]):
+        return False
+    # bf16: torch's float32 -> bf16 on random floats
+    x = np.random.default_rng(7).standard_normal(20000).astype(np.float32)
+    out = np.empty(x.size, np.uint16)
+    lib.dgo_bf16_round(_ptr(x.astype(np.float64)), _ptr(out), x.size)
+    if not np.array_equal(out, torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)):
+        return False
+    # scaled contraction vs float64 matmul of the dequantised inputs
+    p = gi.dense_problem(40, 336, 512, seed_a=21, seed_b=22)
+    sa = np.ascontiguousarray(p["sA"])
+    d64 = np.empty((40, 336), np.float64)
+    d16 = np.empty((40, 336), np.uint16)
+    lib.dgo_gemm_nt(_ptr(np.ascontiguousarray(p["A"])), _ptr(sa), _ptr(np.ascontiguousarray(p["B"])),
+                    _ptr(np.ascontiguousarray(p["sB"])), 40, 336, 512, _ptr(d64), _ptr(d16))
+    a = torch.from_numpy(p["A"]).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    b = torch.from_numpy(p["B"]).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    a = a * np.repeat(sa.astype(np.float64), 128, axis=1)
+    b = b * np.repeat(np.repeat(p["sB"].astype(np.float64), 128, axis=0)[:336], 128, axis=1)
+    bound = np.abs(a) @ np.abs(b).T
+    return bool(np.all(np.abs(d64 - a @ b.T) <= 1e-12 * bound + 1e-300))
+
+
+def test_unmutated_copy_passes(tmp_path):
+    lib = _build_variant(tmp_path, "#define DGO_BLOCK 128", "#define DGO_BLOCK 128")
+    assert _pins_pass(lib)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(tmp_path, name):
+    old, new = MUTATIONS[name]
+    lib = _build_variant(tmp_path, old, new)
+    assert not _pins_pass(lib), f"no pin caught: {name}"
