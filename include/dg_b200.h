@@ -177,6 +177,18 @@ dg_status_t dg_set_num_sms(int n);
 /* SMs the next launch on the current device will use. */
 int dg_get_num_sms(void);
 
+/* Tile families the planner may choose from (process-wide; for tuning and
+ * tests -- the default lets the cost model decide).  One-CTA tiles are
+ * 128 rows on one SM; pair tiles are 256 rows on the two SMs of a cluster
+ * sharing one tcgen05 cta_group::2 MMA.  Forcing pair tiles also lifts the
+ * rule that they are used only when they fill every SM pair.  The K-split
+ * decode path is a one-CTA family.  Returns DG_ERR_INVALID_ARG for any other
+ * value.  (A tuning control of this library; the pages have no counterpart.) */
+#define DG_TILES_AUTO 0
+#define DG_TILES_ONE_CTA 1
+#define DG_TILES_PAIR 2
+dg_status_t dg_set_tile_family(int family);
+
 /* Time limit of each pipeline wait inside the kernels, in nanoseconds
  * (default 2e9).  A wait that runs past it makes the kernel record
  * DG_ERR_TIMEOUT, drain its in-flight copies and return.  0 restores the

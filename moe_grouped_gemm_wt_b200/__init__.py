@@ -46,6 +46,7 @@ _SIGNATURES = {
     "dg_get_tma_aligned_size": (_I, [_I, _I]),
     "dg_set_num_sms": (_I, [_I]),
     "dg_get_num_sms": (_I, []),
+    "dg_set_tile_family": (_I, [_I]),
     "dg_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
     "dg_set_stall_injection": (_I, [_I]),
     "dg_get_device_status": (_I, [_P]),
@@ -134,6 +135,14 @@ def dg_set_num_sms(n: int) -> None:
 
 def dg_get_num_sms() -> int:
     return load_library().dg_get_num_sms()
+
+
+DG_TILES_AUTO, DG_TILES_ONE_CTA, DG_TILES_PAIR = 0, 1, 2
+
+
+def dg_set_tile_family(family: int) -> None:
+    """Restrict the planner to one tile family (DG_TILES_*); 0 = automatic."""
+    _check("dg_set_tile_family", load_library().dg_set_tile_family(family))
 
 
 def dg_set_wait_timeout_ns(ns: int) -> None:

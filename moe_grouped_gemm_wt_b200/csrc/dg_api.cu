@@ -1,6 +1,7 @@
 // dg_api.cu -- host side of the C ABI declared in include/dg_b200.h:
 // argument validation, tile-shape choice, TMA descriptor encoding and kernel
-// launch.  All arithmetic of the GEMM runs in fp8_gemm_kernel.cuh.
+// launch.  All arithmetic of the GEMM runs in fp8_gemm_kernel.cuh (one CTA
+// per tile) and fp8_gemm_pair_kernel.cuh (a CTA pair per 256-row tile).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -12,11 +13,13 @@
 
 #include "../../include/dg_b200.h"
 #include "fp8_gemm_kernel.cuh"
+#include "fp8_gemm_pair_kernel.cuh"
 
 namespace {
 
 using dg::GemmParams;
 using dg::KernelConfig;
+using dg::PairConfig;
 
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
@@ -155,13 +158,15 @@ struct TileChoice {
     int stages;
     int ks;      // 128-wide K blocks per pipeline stage
     int split;   // 0: persistent tiles; 1: K split over a cluster (dense only)
-    double kb_ns;  // measured time of one K block of one tile (cost model)
+    double kb_ns;    // measured time of one K block of one tile (cost model, us)
+    int pair;        // 1: 256 x bn tiles on CTA pairs (cta_group::2)
+    double tile_us;  // per-tile fill, drain and epilogue (cost model, us)
 };
 constexpr TileChoice kTileChoices[] = {
-    {112, 3, 2, 0, 0.41}, {128, 5, 1, 0, 0.53}, {224, 2, 2, 0, 0.78}, {256, 3, 1, 0, 0.68},
-    {144, 3, 2, 1, 0.40},
+    {112, 3, 2, 0, 0.41, 0, 1.9}, {128, 5, 1, 0, 0.53, 0, 1.9}, {224, 2, 2, 0, 0.78, 0, 1.9},
+    {256, 3, 1, 0, 0.68, 0, 1.9}, {144, 3, 2, 1, 0.40, 0, 1.9}, {160, 3, 2, 0, 0.453, 1, 2.2},
+    {192, 3, 2, 0, 0.511, 1, 2.2},
 };
-constexpr int kNumChoices = sizeof(kTileChoices) / sizeof(kTileChoices[0]);
 constexpr int kSplitFixedNs = 1500;  // cluster reduction + pipeline fill of a split CTA
 
 // DG_FORCE_BLOCK_N=<n> pins the tile width to one of the compiled choices
@@ -176,6 +181,33 @@ int forced_block_n()
     return v;
 }
 
+// Tile family restriction (dg_set_tile_family): -1 none, 0 one-CTA tiles
+// only, 1 pair tiles only.  Its initial value comes from DG_FORCE_PAIR=0|1.
+std::atomic<int> g_forced_pair{-2};
+
+int forced_pair()
+{
+    int v = g_forced_pair.load();
+    if (v == -2) {
+        const char *e = std::getenv("DG_FORCE_PAIR");
+        const int init = (e && e[0]) ? (std::atoi(e) != 0 ? 1 : 0) : -1;
+        g_forced_pair.compare_exchange_strong(v, init);
+        v = g_forced_pair.load();
+    }
+    return v;
+}
+
+// DG_PRINT_CONFIGS=1 prints each call's plan to stderr.
+bool print_configs()
+{
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("DG_PRINT_CONFIGS");
+        v = (e && e[0] && e[0] != '0') ? 1 : 0;
+    }
+    return v == 1;
+}
+
 struct Plan {
     TileChoice c;
     int ksplit;  // CTAs per cluster sharing a tile's K range (1 = none)
@@ -187,8 +219,10 @@ int max_active_clusters(const TileChoice &c, int S);
 // "完全JIT设计"; non-power-of-two BLOCK_N to fill the SMs, section
 // "非对齐块大小"): waves of tiles over the SMs times the time of one tile.
 // When a problem has too few tiles to fill the GPU (decode shapes), the K
-// range of each tile may be split over a cluster of 2..16 CTAs.
-Plan choose_plan(int64_t m_blocks, int N, int num_kb, int sms, bool allow_split)
+// range of each tile may be split over a cluster of 2..16 CTAs.  Pair tiles
+// (256 rows on two SMs) are taken only by problems with at least one full
+// wave of them.  m_blocks counts 128-row blocks, pair_rows 256-row ones.
+Plan choose_plan(int64_t m_blocks, int64_t pair_rows, int N, int num_kb, int sms, bool allow_split)
 {
     Plan best{kTileChoices[0], 1};
     double best_cost = 1e300;
@@ -196,10 +230,25 @@ Plan choose_plan(int64_t m_blocks, int N, int num_kb, int sms, bool allow_split)
         const bool forced = forced_block_n() > 0;
         if (forced && c.bn != forced_block_n())
             continue;
+        if (forced_pair() >= 0 && c.pair != forced_pair())
+            continue;
+        if (c.pair) {
+            const int pairs = sms / 2;
+            const int64_t tiles = pair_rows * ((N + c.bn - 1) / c.bn);
+            if (pairs <= 0 || (tiles < pairs && forced_pair() != 1))
+                continue;
+            const int64_t waves = (tiles + pairs - 1) / pairs;
+            const double cost = static_cast<double>(waves) * (num_kb * c.kb_ns + c.tile_us);
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = Plan{c, 1};
+            }
+            continue;
+        }
         const int64_t tiles = m_blocks * ((N + c.bn - 1) / c.bn);
         if (!c.split) {
             const int64_t waves = (tiles + sms - 1) / sms;
-            const double cost = static_cast<double>(waves) * num_kb * c.kb_ns;
+            const double cost = static_cast<double>(waves) * (num_kb * c.kb_ns + c.tile_us);
             if (cost < best_cost) {
                 best_cost = cost;
                 best = Plan{c, 1};
@@ -217,7 +266,7 @@ Plan choose_plan(int64_t m_blocks, int N, int num_kb, int sms, bool allow_split)
                 continue;
             if (tiles > max_active_clusters(c, S))
                 continue;
-            const double cost = kbps * c.kb_ns + kSplitFixedNs * 1e-3;
+            const double cost = kbps * c.kb_ns + c.tile_us + kSplitFixedNs * 1e-3;
             if (cost < best_cost) {
                 best_cost = cost;
                 best = Plan{c, S};
@@ -296,6 +345,69 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
     return DG_OK;
 }
 
+// Pair tiles: a cluster of two CTAs per 256 x BN tile, persistent over
+// tiles; grid = 2 x (pairs in use).
+template <int BN, int STAGES, int KS, int LAYOUT>
+dg_status_t launch_pair(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
+                        const GemmParams &p, int grid, cudaStream_t stream)
+{
+    using Cfg = PairConfig<BN, STAGES, KS>;
+    CUtensorMap ta, tb;
+    if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
+        !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, Cfg::BN_HALF, KS))
+        return DG_ERR_CUDA;
+    // output boxes of 128 rows: 32 columns with 64-byte swizzle, and a
+    // 16-column unswizzled remainder box
+    CUtensorMap tdbox, tdrem;
+    if (!make_tmap_bf16(&tdbox, p.D, static_cast<uint64_t>(p.N), a_rows, Cfg::EPI_BOX, dg::kBM,
+                        CU_TENSOR_MAP_SWIZZLE_64B))
+        return DG_ERR_CUDA;
+    if (Cfg::EPI_REM > 0) {
+        if (!make_tmap_bf16(&tdrem, p.D, static_cast<uint64_t>(p.N), a_rows, Cfg::EPI_REM, dg::kBM,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+            return DG_ERR_CUDA;
+    } else {
+        tdrem = tdbox;
+    }
+    auto kern = dg::fp8_gemm_pair_kernel<BN, STAGES, KS, LAYOUT>;
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices)
+        return DG_ERR_CUDA;
+    if (!attr_set[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::SMEM_BYTES) != cudaSuccess)
+            return DG_ERR_CUDA;
+        attr_set[dev].store(true);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (print_configs()) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            n = -1;
+        }
+        std::fprintf(stderr, "[dg] pair kernel: grid %d CTAs, %d co-resident pairs possible, smem %d B\n",
+                     grid, n, Cfg::SMEM_BYTES);
+    }
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tdbox, tdrem, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DG_ERR_CUDA;
+    }
+    return DG_OK;
+}
+
 // Co-resident clusters of S CTAs of a split configuration (cached per
 // device).  The split kernel keeps one tile per cluster, so a plan is only
 // used when every cluster of the grid fits at once.
@@ -354,6 +466,26 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
 {
     const TileChoice &c = plan.c;
     p.num_nb = (p.N + c.bn - 1) / c.bn;
+    if (c.pair) {
+        // the pair scheduler counts 256-row pair rows
+        p.num_mb = (p.num_mb + 1) / 2;
+        if (LAYOUT != dg::kMasked)
+            p.raster = choose_raster(p.num_mb);
+        p.ksplit = 1;
+        p.kb_per_split = p.num_kb;
+        const int pairs = sms / 2;
+        const int64_t ptiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
+        int grid_pairs = pairs;
+        if (LAYOUT != dg::kMasked && ptiles < pairs)
+            grid_pairs = static_cast<int>(ptiles);
+        if (grid_pairs <= 0)
+            return DG_OK;
+        if (c.bn == 160 && c.stages == 3 && c.ks == 2)
+            return launch_pair<160, 3, 2, LAYOUT>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
+        if (c.bn == 192 && c.stages == 3 && c.ks == 2)
+            return launch_pair<192, 3, 2, LAYOUT>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
+        return DG_ERR_UNSUPPORTED;
+    }
     p.ksplit = plan.ksplit;
     p.kb_per_split = (p.num_kb + plan.ksplit - 1) / plan.ksplit;
     const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
@@ -402,16 +534,6 @@ dg_status_t check_common(const void *A, const float *sA, const void *B, const fl
     return DG_OK;
 }
 
-bool print_configs()
-{
-    static int v = -1;
-    if (v < 0) {
-        const char *e = std::getenv("DG_PRINT_CONFIGS");
-        v = (e && e[0] && e[0] != '0') ? 1 : 0;
-    }
-    return v == 1;
-}
-
 }  // namespace
 
 // =================================================================== C ABI
@@ -447,10 +569,10 @@ dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B, const 
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
     p.stall_injection = g_stall_injection.load();
-    const Plan plan = choose_plan(p.num_mb, N, p.num_kb, sms, true);
+    const Plan plan = choose_plan(p.num_mb, (M + 255) / 256, N, p.num_kb, sms, true);
     if (print_configs())
-        std::fprintf(stderr, "[dg] dense M=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d ksplit=%d sms=%d\n",
-                     M, N, K, plan.c.bn, plan.c.stages, plan.c.ks, plan.ksplit, sms);
+        std::fprintf(stderr, "[dg] dense M=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d ksplit=%d sms=%d\n",
+                     M, N, K, plan.c.pair ? 256 : 128, plan.c.bn, plan.c.stages, plan.c.ks, plan.ksplit, sms);
     return dispatch<dg::kDense>(plan, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), p,
                                 sms, stream);
 }
@@ -493,10 +615,11 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
     p.stall_injection = g_stall_injection.load();
-    const Plan plan = choose_plan(p.num_mb, N, p.num_kb, sms, false);
+    const Plan plan = choose_plan(p.num_mb, (M_total + 255) / 256, N, p.num_kb, sms, false);
     if (print_configs())
-        std::fprintf(stderr, "[dg] contiguous M=%d N=%d K=%d G=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
-                     M_total, N, K, num_groups, plan.c.bn, plan.c.stages, plan.c.ks, sms);
+        std::fprintf(stderr, "[dg] contiguous M=%d N=%d K=%d G=%d -> BM=%d BN=%d stages=%d ks=%d sms=%d\n",
+                     M_total, N, K, num_groups, plan.c.pair ? 256 : 128, plan.c.bn, plan.c.stages,
+                     plan.c.ks, sms);
     return dispatch<dg::kContiguous>(plan, A, static_cast<uint64_t>(M_total), B,
                                      static_cast<uint64_t>(num_groups) * N, p, sms, stream);
 }
@@ -539,12 +662,14 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const voi
     p.timeout_ns = g_timeout_ns.load();
     p.stall_injection = g_stall_injection.load();
     const int em = (expected_m > 0 && expected_m < max_m) ? expected_m : max_m;
-    const Plan plan = choose_plan(static_cast<int64_t>(num_groups) * ((em + 127) / 128), N,
+    const Plan plan = choose_plan(static_cast<int64_t>(num_groups) * ((em + 127) / 128),
+                                  static_cast<int64_t>(num_groups) * ((em + 255) / 256), N,
                                   p.num_kb, sms, false);
     if (print_configs())
         std::fprintf(stderr,
-                     "[dg] masked G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
-                     num_groups, max_m, em, N, K, plan.c.bn, plan.c.stages, plan.c.ks, sms);
+                     "[dg] masked G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d sms=%d\n",
+                     num_groups, max_m, em, N, K, plan.c.pair ? 256 : 128, plan.c.bn, plan.c.stages,
+                     plan.c.ks, sms);
     return dispatch<dg::kMasked>(plan, A, static_cast<uint64_t>(num_groups) * max_m, B,
                                  static_cast<uint64_t>(num_groups) * N, p, sms, stream);
 }
@@ -569,6 +694,14 @@ dg_status_t dg_set_num_sms(int n)
 }
 
 int dg_get_num_sms(void) { return effective_sms(current_device()); }
+
+dg_status_t dg_set_tile_family(int family)
+{
+    if (family < DG_TILES_AUTO || family > DG_TILES_PAIR)
+        return DG_ERR_INVALID_ARG;
+    g_forced_pair.store(family == DG_TILES_AUTO ? -1 : (family == DG_TILES_PAIR ? 1 : 0));
+    return DG_OK;
+}
 
 dg_status_t dg_set_wait_timeout_ns(uint64_t ns)
 {
@@ -619,14 +752,17 @@ int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, i
     if (sms <= 0)
         sms = g_num_sms_cap.load() > 0 ? g_num_sms_cap.load() : 148;
     int64_t m_blocks = (M + 127) / 128;
-    if (layout == 2)
+    int64_t pair_rows = (M + 255) / 256;
+    if (layout == 2) {
         m_blocks *= groups;
-    const Plan plan = choose_plan(m_blocks, N, K / 128 > 0 ? K / 128 : 1, sms, layout == 0);
+        pair_rows *= groups;
+    }
+    const Plan plan = choose_plan(m_blocks, pair_rows, N, K / 128 > 0 ? K / 128 : 1, sms, layout == 0);
     const TileChoice &c = plan.c;
     return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
-                         "layout=%d BM=128 BN=%d BK=128 stages=%d ks=%d ksplit=%d sms=%d m_blocks=%lld n_blocks=%d",
-                         layout, c.bn, c.stages, c.ks, plan.ksplit, sms,
-                         static_cast<long long>(m_blocks), (N + c.bn - 1) / c.bn);
+                         "layout=%d BM=%d BN=%d BK=128 stages=%d ks=%d ksplit=%d pair=%d sms=%d m_blocks=%lld n_blocks=%d",
+                         layout, c.pair ? 256 : 128, c.bn, c.stages, c.ks, plan.ksplit, c.pair, sms,
+                         static_cast<long long>(c.pair ? pair_rows : m_blocks), (N + c.bn - 1) / c.bn);
 }
 
 const char *dg_status_string(dg_status_t status)
@@ -731,7 +867,7 @@ extern "C" dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, co
     p.timeout_ns = g_timeout_ns.load();
     p.stall_injection = g_stall_injection.load();
     const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
-    const Plan plan = choose_plan(p.num_mb, N, p.num_kb, sms, true);
+    const Plan plan = choose_plan(p.num_mb, (M + 255) / 256, N, p.num_kb, sms, true);
     int S = 1;
     if (plan.c.split && plan.c.bn == kBN) {
         S = plan.ksplit;

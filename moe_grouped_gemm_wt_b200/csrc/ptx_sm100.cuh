@@ -74,6 +74,11 @@ __device__ __forceinline__ void st_shared_cluster_v4f(uint32_t addr, float4 v)
                  : "memory");
 }
 
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr)
 {
     float4 v;
@@ -113,6 +118,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
+}
+
+// Arrives on a barrier given by its shared::cluster address (a barrier of
+// this CTA or of another CTA of the cluster, from map_shared_rank), with the
+// default semantics (release, CTA scope).  Used to hand a TMEM buffer back:
+// the order against this thread's earlier tcgen05.ld comes from
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync, so no cluster-
+// scope release (a full fence, measured at several hundred cycles) is needed.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 // True once the phase with parity `parity` has completed.
@@ -157,6 +173,20 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// 3-D tiled load for a CTA pair (cta_group::2): the box lands in this CTA's
+// shared memory at `dst`, and its transaction bytes are signalled on
+// `bar_cluster`, a barrier of either CTA of the pair given by its
+// shared::cluster address.  No multicast: one destination, one source.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void *tmap,
+                                                 uint32_t bar_cluster, int x, int y, int z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
 
@@ -241,6 +271,12 @@ __device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t count, b
     return out != 0;
 }
 
+// Waits until every cp.async copy issued by this thread has landed.
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Arrives on `bar` once all earlier cp.async copies of this thread have
 // landed.  .noinc: the arrival is one of the barrier's expected arrivals.
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar)
@@ -270,6 +306,26 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
                  : "memory");
 }
 
+// The same three for a CTA pair (cta_group::2): one warp of EACH CTA of the
+// pair executes them; the pair's MMAs may then write both CTAs' TMEM.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_alloc_permit_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before_sync()
 {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -290,6 +346,34 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uin
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Pair MMA (cta_group::2, M = 256), issued by one thread of the pair's
+// rank-0 CTA: rows 0-127 of A come from rank 0's shared memory and rows
+// 128-255 from rank 1's, B's first N/2 rows from rank 0 and the rest from
+// rank 1, all at the same shared-memory offsets; each CTA's TMEM receives
+// its own 128 rows of D, all N columns.
+__device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives once on the barrier at shared-memory offset `bar` in every CTA of
+// `cta_mask` when all pair MMAs previously issued by this thread have
+// completed (an arrive, not a data load: no multicast copy is involved).
+__device__ __forceinline__ void mma_commit_pair_multicast(uint32_t bar, uint16_t cta_mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar),
+        "h"(cta_mask)
         : "memory");
 }
 
