@@ -161,11 +161,12 @@ struct TileChoice {
     double kb_ns;    // measured time of one K block of one tile (cost model, us)
     int pair;        // 1: 256 x bn tiles on CTA pairs (cta_group::2)
     double tile_us;  // per-tile fill, drain and epilogue (cost model, us)
+    int wg = 2;      // promotion warpgroups (pair tiles: 2 or 3)
 };
 constexpr TileChoice kTileChoices[] = {
     {112, 3, 2, 0, 0.41, 0, 1.9}, {128, 5, 1, 0, 0.53, 0, 1.9}, {224, 2, 2, 0, 0.78, 0, 1.9},
-    {256, 3, 1, 0, 0.68, 0, 1.9}, {144, 3, 2, 1, 0.40, 0, 1.9}, {160, 3, 2, 0, 0.453, 1, 2.2},
-    {192, 3, 2, 0, 0.511, 1, 2.2},
+    {256, 3, 1, 0, 0.68, 0, 1.9}, {144, 3, 2, 1, 0.40, 0, 1.9}, {160, 3, 2, 0, 0.441, 1, 2.2},
+    {192, 3, 2, 0, 0.50, 1, 2.2, 3},
 };
 constexpr int kSplitFixedNs = 1500;  // cluster reduction + pipeline fill of a split CTA
 
@@ -347,11 +348,11 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
 
 // Pair tiles: a cluster of two CTAs per 256 x BN tile, persistent over
 // tiles; grid = 2 x (pairs in use).
-template <int BN, int STAGES, int KS, int LAYOUT>
+template <int BN, int STAGES, int KS, int LAYOUT, int NWG>
 dg_status_t launch_pair(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
                         const GemmParams &p, int grid, cudaStream_t stream)
 {
-    using Cfg = PairConfig<BN, STAGES, KS>;
+    using Cfg = PairConfig<BN, STAGES, KS, NWG>;
     CUtensorMap ta, tb;
     if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
         !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, Cfg::BN_HALF, KS))
@@ -369,7 +370,7 @@ dg_status_t launch_pair(const void *A, uint64_t a_rows, const void *B, uint64_t 
     } else {
         tdrem = tdbox;
     }
-    auto kern = dg::fp8_gemm_pair_kernel<BN, STAGES, KS, LAYOUT>;
+    auto kern = dg::fp8_gemm_pair_kernel<BN, STAGES, KS, LAYOUT, NWG>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices)
@@ -378,6 +379,17 @@ dg_status_t launch_pair(const void *A, uint64_t a_rows, const void *B, uint64_t 
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg::SMEM_BYTES) != cudaSuccess)
             return DG_ERR_CUDA;
+        if (Cfg::REBALANCE) {
+            // setmaxnreg moves registers between warpgroups inside the
+            // block's launch allocation; if the compiled kernel were launched
+            // with fewer registers than the budgets add up to, the increase
+            // would wait forever, so such a build is refused here.
+            cudaFuncAttributes fa{};
+            if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+                return DG_ERR_CUDA;
+            if (fa.numRegs < Cfg::LAUNCH_REGS)
+                return DG_ERR_UNSUPPORTED;
+        }
         attr_set[dev].store(true);
     }
     cudaLaunchConfig_t cfg = {};
@@ -480,10 +492,10 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
             grid_pairs = static_cast<int>(ptiles);
         if (grid_pairs <= 0)
             return DG_OK;
-        if (c.bn == 160 && c.stages == 3 && c.ks == 2)
-            return launch_pair<160, 3, 2, LAYOUT>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
-        if (c.bn == 192 && c.stages == 3 && c.ks == 2)
-            return launch_pair<192, 3, 2, LAYOUT>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
+        if (c.bn == 160 && c.stages == 3 && c.ks == 2 && c.wg == 2)
+            return launch_pair<160, 3, 2, LAYOUT, 2>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
+        if (c.bn == 192 && c.stages == 3 && c.ks == 2 && c.wg == 3)
+            return launch_pair<192, 3, 2, LAYOUT, 3>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
         return DG_ERR_UNSUPPORTED;
     }
     p.ksplit = plan.ksplit;
@@ -760,8 +772,8 @@ int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, i
     const Plan plan = choose_plan(m_blocks, pair_rows, N, K / 128 > 0 ? K / 128 : 1, sms, layout == 0);
     const TileChoice &c = plan.c;
     return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
-                         "layout=%d BM=%d BN=%d BK=128 stages=%d ks=%d ksplit=%d pair=%d sms=%d m_blocks=%lld n_blocks=%d",
-                         layout, c.pair ? 256 : 128, c.bn, c.stages, c.ks, plan.ksplit, c.pair, sms,
+                         "layout=%d BM=%d BN=%d BK=128 stages=%d ks=%d ksplit=%d pair=%d wg=%d sms=%d m_blocks=%lld n_blocks=%d",
+                         layout, c.pair ? 256 : 128, c.bn, c.stages, c.ks, plan.ksplit, c.pair, c.wg, sms,
                          static_cast<long long>(c.pair ? pair_rows : m_blocks), (N + c.bn - 1) / c.bn);
 }
 

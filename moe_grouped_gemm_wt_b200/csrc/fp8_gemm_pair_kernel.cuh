@@ -125,20 +125,35 @@ struct PairScheduler {
     }
 };
 
-template <int BN_, int STAGES_, int KS_>
+// NWG promotion warpgroups split the tile's columns (BN / NWG each).  With
+// three, every promotion thread holds 64 columns and loads its whole partial
+// from TMEM in one round, so each buffer goes back to the MMA early; the
+// block is then 16 warps (three promotion warpgroups and one control
+// warpgroup: the two producers, the MMA warp and one idle warp), launched at
+// 128 registers a thread and rebalanced with setmaxnreg: 152 for each
+// promotion thread, 56 for the control warpgroup.
+template <int BN_, int STAGES_, int KS_, int NWG_ = 2>
 struct PairConfig {
     static constexpr int BN = BN_;          // columns of the pair tile
     static constexpr int BN_HALF = BN / 2;  // B rows held by each CTA
     static constexpr int STAGES = STAGES_;
     static constexpr int KS = KS_;
-    static constexpr int NUM_WG = 2;        // promotion warpgroups, each BN/2 columns
+    static constexpr int NUM_WG = NWG_;     // promotion warpgroups
     static constexpr int BN_WG = BN / NUM_WG;
     static constexpr int RMAX = BN_WG <= 64 ? BN_WG : 32;
     static constexpr int NUM_PROMO_WARPS = 4 * NUM_WG;
     static constexpr int PRODUCER_A_WARP = NUM_PROMO_WARPS;
     static constexpr int PRODUCER_B_WARP = NUM_PROMO_WARPS + 1;
     static constexpr int MMA_WARP = NUM_PROMO_WARPS + 2;
-    static constexpr int THREADS = (NUM_PROMO_WARPS + 3) * 32;
+    static constexpr bool REBALANCE = NUM_WG == 3;
+    static constexpr int CTRL_WARPS = REBALANCE ? 4 : 3;
+    static constexpr int THREADS = (NUM_PROMO_WARPS + CTRL_WARPS) * 32;
+    static constexpr int LAUNCH_REGS = REBALANCE ? 65536 / THREADS : 0;
+    static constexpr int PROMO_REGS = 152;
+    static constexpr int CTRL_REGS = 56;
+    // Warpgroup columns start at multiples of BN_WG; when BN_WG divides 128
+    // they never straddle a 128-wide weight block, so one scale serves them.
+    static constexpr bool UNIFORM_SCALE = (128 % (BN / NWG_) == 0) && (BN % (BN / NWG_) == 0);
     static constexpr int A_BYTES = kBM * kBK;      // one K block of this CTA's A rows
     static constexpr int B_BYTES = BN_HALF * kBK;  // one K block of this CTA's B rows
     static constexpr int STAGE_BYTES = KS * (A_BYTES + B_BYTES);
@@ -160,6 +175,10 @@ struct PairConfig {
     static constexpr int SMEM_BYTES = 1024 /*align slack*/ + EPI_OFFSET + NUM_WG * EPI_WG_BYTES;
 
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair MMA N (M = 256): multiple of 32 up to 256");
+    static_assert(BN % NUM_WG == 0 && (NUM_WG == 2 || NUM_WG == 3), "promotion warpgroups");
+    static_assert(!REBALANCE || (NUM_WG * 128 * PROMO_REGS + 128 * CTRL_REGS <= THREADS * LAUNCH_REGS &&
+                                 LAUNCH_REGS % 8 == 0),
+                  "setmaxnreg budgets must fit the registers the block is launched with");
     static_assert(BN_WG % 16 == 0 && BN_WG <= 128, "promotion columns per warpgroup");
     static_assert(B_BYTES % 1024 == 0, "B tiles must keep 1024-byte swizzle atoms aligned");
     static_assert(NBUF >= 2, "double-buffered TMEM at least");
@@ -183,14 +202,14 @@ __device__ __forceinline__ bool pair_warp_wait(uint32_t bar, uint32_t parity, ui
     return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
-template <int BN, int STAGES, int KS, int LAYOUT>
-__global__ void __launch_bounds__(PairConfig<BN, STAGES, KS>::THREADS, 1)
+template <int BN, int STAGES, int KS, int LAYOUT, int NWG>
+__global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG>::THREADS, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                          const __grid_constant__ CUtensorMap tmap_b,
                          const __grid_constant__ CUtensorMap tmap_dbox,
                          const __grid_constant__ CUtensorMap tmap_drem, const GemmParams p)
 {
-    using Cfg = PairConfig<BN, STAGES, KS>;
+    using Cfg = PairConfig<BN, STAGES, KS, NWG>;
     constexpr int BN_WG = Cfg::BN_WG;
     constexpr int RMAX = Cfg::RMAX;
     constexpr int NBUF = Cfg::NBUF;
@@ -257,6 +276,11 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS>::THREADS, 1)
     const uint32_t full_leader = map_shared_rank(smem_addr(full_bar), 0);
     const uint32_t tempty_leader = map_shared_rank(smem_addr(tempty_bar), 0);
 
+    if (warp >= Cfg::NUM_PROMO_WARPS) {
+    // The control warps.  With REBALANCE, the whole control warpgroup gives
+    // registers up here, at one point that dominates all of its code.
+    if constexpr (Cfg::REBALANCE)
+        setmaxnreg_dec<Cfg::CTRL_REGS>();
     if (warp == Cfg::PRODUCER_A_WARP || warp == Cfg::PRODUCER_B_WARP) {
         // ------------------------------------------------------ TMA producers
         // Warp A: this CTA's A box per stage, plus cp.async copies of the
@@ -399,8 +423,11 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS>::THREADS, 1)
                 wait_bounded(last_bar, last_parity, drain_tmo, abort_flag, kRoleDrain, 32, false);
             __syncwarp();
         }
+    }
     } else {
         // ------------------------------------------------ promotion warps
+        if constexpr (Cfg::REBALANCE)
+            setmaxnreg_inc<Cfg::PROMO_REGS>();
         const int wg = warp / 4;
         const int quad = warp % 4;
         const int row = quad * 32 + lane;  // row within this CTA's half == TMEM lane
@@ -495,10 +522,13 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS>::THREADS, 1)
 #pragma unroll
                         for (int g8 = 0; g8 < RMAX; g8 += 8) {
                             if (whole || g8 < TAIL) {
-                                const float sc = (c0 + g8 >= boundary) ? s_hi[q] : s_lo[q];
+                                // a warpgroup whose columns never straddle a
+                                // 128-wide weight block uses one scale
+                                const float sc = (Cfg::UNIFORM_SCALE || c0 + g8 < boundary) ? s_lo[q] : s_hi[q];
 #pragma unroll
-                                for (int i = 0; i < 8; ++i)
-                                    acc[c0 + g8 + i] = fmaf(__uint_as_float(r[g8 + i]), sc, acc[c0 + g8 + i]);
+                                for (int i = 0; i < 8; i += 2)
+                                    fma2_rn(acc[c0 + g8 + i], acc[c0 + g8 + i + 1], __uint_as_float(r[g8 + i]),
+                                            __uint_as_float(r[g8 + i + 1]), sc);
                             }
                         }
                     }

@@ -284,6 +284,41 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar)
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// ------------------------------------------------------------------ FP32
+
+// (d0, d1) = (a0 * s + d0, a1 * s + d1): two independent round-to-nearest
+// fp32 FMAs in one packed instruction (fma.rn.f32x2), bit-identical to two
+// fmaf calls; it halves the instructions of the promotion loop.
+__device__ __forceinline__ void fma2_rn(float &d0, float &d1, float a0, float a1, float s)
+{
+    asm("{\n\t.reg .b64 d, a, m;\n\t"
+        "mov.b64 d, {%0, %1};\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 m, {%4, %4};\n\t"
+        "fma.rn.f32x2 d, a, m, d;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "+f"(d0), "+f"(d1)
+        : "f"(a0), "f"(a1), "f"(s));
+}
+
+// ------------------------------------------------------------- registers
+
+// Per-warpgroup register budgets (all four warps of a warpgroup execute
+// these).  The block keeps the total it was launched with: the sum of the
+// budgets over its warpgroups must not exceed threads x launch registers,
+// or an increase waits forever; callers check that before launching.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------- tcgen05
 
 // Allocates `ncols` TMEM columns (power of two >= 32); the base address is
