@@ -268,8 +268,14 @@ struct KernelConfig {
     static constexpr int EPI_WG_BYTES = kBM * 128;  // 128 rows x 128 bytes
     static constexpr int PIPE_BYTES = STAGES * (STAGE_BYTES + SA_BYTES + SB_BYTES);
     static constexpr int EPI_OFFSET = (PIPE_BYTES + BAR_BYTES + 1023) / 1024 * 1024;
+    // One staging buffer per output box when shared memory allows, so a
+    // warpgroup stores all its boxes without waiting for an earlier store to
+    // finish reading its buffer; else one buffer reused box after box.
+    static constexpr int EPI_BOXES = EPI_FULL_BOXES + (EPI_REM > 0 ? 1 : 0);
+    static constexpr int EPI_BUFS =
+        1024 + EPI_OFFSET + NUM_WG * EPI_BOXES * EPI_WG_BYTES <= 232448 ? EPI_BOXES : 1;
     static constexpr int SMEM_BYTES =
-        1024 /*align slack*/ + EPI_OFFSET + (SPLIT ? 0 : NUM_WG * EPI_WG_BYTES);
+        1024 /*align slack*/ + EPI_OFFSET + (SPLIT ? 0 : NUM_WG * EPI_BUFS * EPI_WG_BYTES);
 
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128: multiple of 16, <= 256");
     static_assert(BN_WG % 8 == 0, "promotion columns per warpgroup must be a multiple of 8");
@@ -340,7 +346,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
     uint64_t *tempty_bar = bars + 3 * STAGES + NBUF;  // TMEM partial buffer read out
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 2 * NBUF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    uint8_t *epi_stage = smem + Cfg::EPI_OFFSET;  // 1024-byte aligned, one buffer per warpgroup
+    uint8_t *epi_stage = smem + Cfg::EPI_OFFSET;  // 1024-byte aligned, EPI_BUFS buffers per warpgroup
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -662,18 +668,20 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                 1 + wg, 128, LAYOUT == kDense ? (tc.mb * kBM < p.M) : row_ok);
             if (tile_rows_ok) {
                 const int grow0 = (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * kBM;
-                const uint32_t stg = smem_addr(epi_stage + wg * Cfg::EPI_WG_BYTES);
 #pragma unroll
-                for (int bx = 0; bx < Cfg::EPI_FULL_BOXES + (Cfg::EPI_REM > 0 ? 1 : 0); ++bx) {
+                for (int bx = 0; bx < Cfg::EPI_BOXES; ++bx) {
                     const bool full = bx < Cfg::EPI_FULL_BOXES;
                     const int cbase = bx * 64;
                     const int ncols = full ? 64 : Cfg::EPI_REM;
                     if (col0 + cbase >= p.N)
                         break;  // this box (and any after it) lies past N
-                    // the previous store from this staging buffer must have
-                    // finished reading it before it is overwritten
+                    const uint32_t stg =
+                        smem_addr(epi_stage + (wg * Cfg::EPI_BUFS + bx % Cfg::EPI_BUFS) * Cfg::EPI_WG_BYTES);
+                    // the store that last used this staging buffer (one per
+                    // box, the most recent EPI_BUFS - 1 may still be pending)
+                    // must have finished reading it before it is overwritten
                     if (wg_tid == 0)
-                        bulk_wait_group_read<0>();
+                        bulk_wait_group_read<Cfg::EPI_BUFS - 1>();
                     named_barrier_sync(1 + wg, 128);
 #pragma unroll
                     for (int ch = 0; ch < 8; ++ch) {

@@ -172,7 +172,12 @@ struct PairConfig {
     static constexpr int EPI_WG_BYTES = kBM * EPI_BOX * 2;
     static constexpr int PIPE_BYTES = STAGES * (STAGE_BYTES + SA_BYTES + SB_BYTES);
     static constexpr int EPI_OFFSET = (PIPE_BYTES + BAR_BYTES + 1023) / 1024 * 1024;
-    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + EPI_OFFSET + NUM_WG * EPI_WG_BYTES;
+    // One staging buffer per output box when shared memory allows (as in the
+    // one-CTA kernel), else one buffer reused box after box.
+    static constexpr int EPI_BOXES = EPI_FULL_BOXES + (EPI_REM > 0 ? 1 : 0);
+    static constexpr int EPI_BUFS =
+        1024 + EPI_OFFSET + NUM_WG * EPI_BOXES * EPI_WG_BYTES <= 232448 ? EPI_BOXES : 1;
+    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + EPI_OFFSET + NUM_WG * EPI_BUFS * EPI_WG_BYTES;
 
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair MMA N (M = 256): multiple of 32 up to 256");
     static_assert(BN % NUM_WG == 0 && (NUM_WG == 2 || NUM_WG == 3), "promotion warpgroups");
@@ -230,7 +235,7 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG>::THREADS, 1)
     uint64_t *tempty_bar = bars + 4 * STAGES + NBUF;  // (leader) both CTAs read the buffer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 2 * NBUF);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    uint8_t *epi_stage = smem + Cfg::EPI_OFFSET;  // 1024-byte aligned, one buffer per warpgroup
+    uint8_t *epi_stage = smem + Cfg::EPI_OFFSET;  // 1024-byte aligned, EPI_BUFS buffers per warpgroup
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -551,16 +556,17 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG>::THREADS, 1)
                 1 + wg, 128, LAYOUT == kDense ? (m_half < p.M) : row_ok);
             if (tile_rows_ok) {
                 const int grow0 = (LAYOUT == kMasked ? tc.g * p.M : 0) + m_half;
-                const uint32_t stg = smem_addr(epi_stage + wg * Cfg::EPI_WG_BYTES);
 #pragma unroll
-                for (int bx = 0; bx < Cfg::EPI_FULL_BOXES + (Cfg::EPI_REM > 0 ? 1 : 0); ++bx) {
+                for (int bx = 0; bx < Cfg::EPI_BOXES; ++bx) {
                     const bool full = bx < Cfg::EPI_FULL_BOXES;
                     const int cbase = bx * Cfg::EPI_BOX;
                     const int ncols = full ? Cfg::EPI_BOX : Cfg::EPI_REM;
                     if (col0 + cbase >= p.N)
                         break;  // this box (and any after it) lies past N
+                    const uint32_t stg =
+                        smem_addr(epi_stage + (wg * Cfg::EPI_BUFS + bx % Cfg::EPI_BUFS) * Cfg::EPI_WG_BYTES);
                     if (wg_tid == 0)
-                        bulk_wait_group_read<0>();
+                        bulk_wait_group_read<Cfg::EPI_BUFS - 1>();
                     named_barrier_sync(1 + wg, 128);
 #pragma unroll
                     for (int ch = 0; ch < Cfg::EPI_BOX / 8; ++ch) {
