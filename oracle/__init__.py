@@ -17,6 +17,9 @@ Parity status of each function (what pins it is listed in the tests):
                                 (exact with unit scales, 1e-12 with scales),
                                 integer inputs, identity/zero, power-of-two
                                 invariance, brute-force loops on tiny cases
+  gemm_nt_acc (+ _sampled)      pinned: integer inputs plus an integer C
+                                (exact), C alone (A = 0), the closed form
+                                C + float64 matmul, numpy's double->float32
   grouped_contiguous / masked   pinned: per-group dense results, placement,
                                 untouched padding / masked rows
   fp32_promotion_sampled        analysis aid (not a reference), pinned against
@@ -67,6 +70,10 @@ def _load():
         lib.dgo_bf16_round.argtypes = [P, P, I64]
         lib.dgo_gemm_nt.restype = I
         lib.dgo_gemm_nt.argtypes = [P, P, P, P, I, I, I, P, P]
+        lib.dgo_gemm_nt_acc.restype = I
+        lib.dgo_gemm_nt_acc.argtypes = [P, P, P, P, P, I, I, I, P, P]
+        lib.dgo_gemm_nt_acc_sampled.restype = I
+        lib.dgo_gemm_nt_acc_sampled.argtypes = [P, P, P, P, P, I, I, I, P, P, I64, P, P]
         lib.dgo_gemm_nt_sampled.restype = I
         lib.dgo_gemm_nt_sampled.argtypes = [P, P, P, P, I, I, I, P, P, I64, P, P]
         lib.dgo_grouped_contiguous.restype = I
@@ -159,6 +166,42 @@ def gemm_nt_sampled(A, sA, B, sB, rows, cols):
     if rc:
         raise ValueError("dgo_gemm_nt_sampled: bad sizes or indices")
     return o64, o16
+
+
+def gemm_nt_acc(A, sA, B, sB, C, want_f64: bool = True):
+    """Dense D = C + A @ B.T with C, D float32 [M][N] (sum in double, one
+    rounding to float32).  Returns (D64 or None, D32)."""
+    A, B, sA, sB = _u8(A), _u8(B), _f32(sA), _f32(sB)
+    C = _f32(C)
+    M, K = A.shape
+    N = B.shape[0]
+    assert B.shape[1] == K and sA.shape == (M, K // BLOCK) and C.shape == (M, N)
+    assert sB.shape == ((N + BLOCK - 1) // BLOCK, K // BLOCK)
+    d64 = np.empty((M, N), dtype=np.float64) if want_f64 else None
+    d32 = np.empty((M, N), dtype=np.float32)
+    rc = _load().dgo_gemm_nt_acc(_ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(C), M, N, K,
+                                 _ptr(d64), _ptr(d32))
+    if rc:
+        raise ValueError("dgo_gemm_nt_acc: bad sizes")
+    return d64, d32
+
+
+def gemm_nt_acc_sampled(A, sA, B, sB, C, rows, cols):
+    """gemm_nt_acc at the (rows[i], cols[i]) pairs: (f64 values, float32)."""
+    A, B, sA, sB = _u8(A), _u8(B), _f32(sA), _f32(sB)
+    C = _f32(C)
+    M, K = A.shape
+    N = B.shape[0]
+    assert C.shape == (M, N)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    cols = np.ascontiguousarray(cols, dtype=np.int64)
+    o64 = np.empty(rows.shape, dtype=np.float64)
+    o32 = np.empty(rows.shape, dtype=np.float32)
+    rc = _load().dgo_gemm_nt_acc_sampled(_ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(C), M, N, K,
+                                         _ptr(rows), _ptr(cols), rows.size, _ptr(o64), _ptr(o32))
+    if rc:
+        raise ValueError("dgo_gemm_nt_acc_sampled: bad sizes or indices")
+    return o64, o32
 
 
 def fp32_promotion_sampled(A, sA, B, sB, rows, cols):

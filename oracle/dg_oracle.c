@@ -179,6 +179,65 @@ int dgo_gemm_nt(const uint8_t *A, const float *sA, const uint8_t *B,
     return 0;
 }
 
+/* Dense NT with an accumulator: D = C + A.B^T, the "D = C + A @ B" form of
+ * the hada.io page (section "Giao dien GEMM va rang buoc layout", where
+ * fp8_gemm_nt computes D = C + A @ B.T).  The page gives C no type; here C
+ * and D are fp32 [M][N] (the reading for accumulating into an fp32 buffer,
+ * C may be the buffer D itself).  C[m,n] plus the exact double result of
+ * dgo_gemm_nt is rounded once from double to fp32 (round to nearest even,
+ * the C conversion under the default rounding mode). */
+int dgo_gemm_nt_acc(const uint8_t *A, const float *sA, const uint8_t *B,
+                    const float *sB, const float *C, int M, int N, int K,
+                    double *D64, float *D32)
+{
+    if (dgo_check_dims(M, N, K) || !C)
+        return -1;
+    dgo_init_lut();
+    int nkb = K / DGO_BLOCK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int m = 0; m < M; ++m) {
+        for (int n = 0; n < N; ++n) {
+            double v = (double)C[(int64_t)m * N + n] +
+                       dgo_element(A + (int64_t)m * K, sA + (int64_t)m * nkb,
+                                   B + (int64_t)n * K,
+                                   sB + (int64_t)(n / DGO_BLOCK) * nkb, K);
+            if (D64)
+                D64[(int64_t)m * N + n] = v;
+            if (D32)
+                D32[(int64_t)m * N + n] = (float)v;
+        }
+    }
+    return 0;
+}
+
+/* dgo_gemm_nt_acc at selected (row, col) pairs; C is the whole [M][N]
+ * accumulator. */
+int dgo_gemm_nt_acc_sampled(const uint8_t *A, const float *sA, const uint8_t *B,
+                            const float *sB, const float *C, int M, int N, int K,
+                            const int64_t *rows, const int64_t *cols, int64_t count,
+                            double *out64, float *out32)
+{
+    if (dgo_check_dims(M, N, K) || !C)
+        return -1;
+    dgo_init_lut();
+    int nkb = K / DGO_BLOCK;
+    for (int64_t i = 0; i < count; ++i)
+        if (rows[i] < 0 || rows[i] >= M || cols[i] < 0 || cols[i] >= N)
+            return -1;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t i = 0; i < count; ++i) {
+        int64_t m = rows[i], n = cols[i];
+        double v = (double)C[m * N + n] +
+                   dgo_element(A + m * K, sA + m * nkb, B + n * K,
+                               sB + (n / DGO_BLOCK) * nkb, K);
+        if (out64)
+            out64[i] = v;
+        if (out32)
+            out32[i] = (float)v;
+    }
+    return 0;
+}
+
 /* Dense NT at selected (row, col) pairs only, for problems too large to
  * compute whole.  Same layouts as dgo_gemm_nt. */
 int dgo_gemm_nt_sampled(const uint8_t *A, const float *sA, const uint8_t *B,

@@ -21,11 +21,11 @@ SRC = os.path.join(ROOT, "oracle", "dg_oracle.c")
 
 MUTATIONS = {
     "weight-block index n%128 instead of n/128": (
-        "sB + (int64_t)(n / DGO_BLOCK) * nkb, K);\n            if (D64)\n                D64[(int64_t)m * N + n] = v;",
-        "sB + (int64_t)(n % DGO_BLOCK) * nkb, K);\n            if (D64)\n                D64[(int64_t)m * N + n] = v;"),
+        "            double v = dgo_element(A + (int64_t)m * K, sA + (int64_t)m * nkb,\n                                   B + (int64_t)n * K,\n                                   sB + (int64_t)(n / DGO_BLOCK) * nkb, K);",
+        "            double v = dgo_element(A + (int64_t)m * K, sA + (int64_t)m * nkb,\n                                   B + (int64_t)n * K,\n                                   sB + (int64_t)(n % DGO_BLOCK) * nkb, K);"),
     "B row stride 1 instead of K (transposed operand)": (
-        "                                   B + (int64_t)n * K,\n                                   sB + (int64_t)(n / DGO_BLOCK) * nkb, K);\n            if (D64)\n                D64[(int64_t)m * N + n] = v;",
-        "                                   B + (int64_t)n,\n                                   sB + (int64_t)(n / DGO_BLOCK) * nkb, K);\n            if (D64)\n                D64[(int64_t)m * N + n] = v;"),
+        "            double v = dgo_element(A + (int64_t)m * K, sA + (int64_t)m * nkb,\n                                   B + (int64_t)n * K,\n",
+        "            double v = dgo_element(A + (int64_t)m * K, sA + (int64_t)m * nkb,\n                                   B + (int64_t)n,\n"),
     "first K block dropped": (
         "    for (int kb = 0; kb < nkb; ++kb) {\n        double partial = 0.0;\n        for (int k = kb * DGO_BLOCK; k < (kb + 1) * DGO_BLOCK; ++k)\n            partial += g_lut[a_row[k]] * g_lut[b_row[k]];\n        double scale",
         "    for (int kb = 1; kb < nkb; ++kb) {\n        double partial = 0.0;\n        for (int k = kb * DGO_BLOCK; k < (kb + 1) * DGO_BLOCK; ++k)\n            partial += g_lut[a_row[k]] * g_lut[b_row[k]];\n        double scale"),
@@ -38,6 +38,9 @@ MUTATIONS = {
     "bf16 truncation instead of round-to-nearest-even": (
         "double nq = nearbyint(r);",
         "double nq = floor(r);"),
+    "accumulator C dropped from D = C + A.B^T": (
+        "            double v = (double)C[(int64_t)m * N + n] +\n                       dgo_element(",
+        "            double v = 0.0 * (double)C[(int64_t)m * N + n] +\n                       dgo_element("),
 }
 
 
@@ -55,6 +58,8 @@ def _build_variant(tmp_path, old, new):
     lib.dgo_gemm_nt.restype = I
     lib.dgo_decode_e4m3.argtypes = [P, P, I64]
     lib.dgo_bf16_round.argtypes = [P, P, I64]
+    lib.dgo_gemm_nt_acc.argtypes = [P, P, P, P, P, I, I, I, P, P]
+    lib.dgo_gemm_nt_acc.restype = I
     return lib
 
 
@@ -90,7 +95,20 @@ def _pins_pass(lib) -> bool:
     a = a * np.repeat(sa.astype(np.float64), 128, axis=1)
     b = b * np.repeat(np.repeat(p["sB"].astype(np.float64), 128, axis=0)[:336], 128, axis=1)
     bound = np.abs(a) @ np.abs(b).T
-    return bool(np.all(np.abs(d64 - a @ b.T) <= 1e-12 * bound + 1e-300))
+    if not np.all(np.abs(d64 - a @ b.T) <= 1e-12 * bound + 1e-300):
+        return False
+    # accumulate form: integer inputs and an integer C, exact
+    rng = np.random.default_rng(8)
+    ai, bi = rng.integers(-4, 5, (8, 256)), rng.integers(-4, 5, (128, 256))
+    ci = rng.integers(-1000, 1001, (8, 128)).astype(np.float32)
+    to8 = lambda x: torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    a8, b8 = np.ascontiguousarray(to8(ai)), np.ascontiguousarray(to8(bi))
+    ones_a, ones_b = np.ones((8, 2), np.float32), np.ones((1, 2), np.float32)
+    e64 = np.empty((8, 128), np.float64)
+    e32 = np.empty((8, 128), np.float32)
+    lib.dgo_gemm_nt_acc(_ptr(a8), _ptr(ones_a), _ptr(b8), _ptr(ones_b), _ptr(ci), 8, 128, 256,
+                        _ptr(e64), _ptr(e32))
+    return bool(np.array_equal(e64, (ci + ai @ bi.T).astype(np.float64)))
 
 
 def test_unmutated_copy_passes(tmp_path):

@@ -186,6 +186,55 @@ def test_sampled_matches_full(oracle_mod):
     assert np.array_equal(s16, d16[r, c])
 
 
+# ------------------------------------------------------ D = C + A @ B.T
+
+def test_acc_integer_inputs_and_integer_c_exact(oracle_mod):
+    # integer-valued e4m3, unit scales and an integer C: every sum is an
+    # integer below 2^24, so the float32 result is exact
+    rng = np.random.default_rng(15)
+    M, N, K = 36, 144, 384
+    ai = rng.integers(-4, 5, (M, K))
+    bi = rng.integers(-4, 5, (N, K))
+    ci = rng.integers(-100000, 100001, (M, N))
+    a = torch.from_numpy(ai.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    b = torch.from_numpy(bi.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    sa = np.ones((M, K // BLOCK), np.float32)
+    sb = np.ones(((N + 127) // 128, K // BLOCK), np.float32)
+    d64, d32 = oracle_mod.gemm_nt_acc(a, sa, b, sb, ci.astype(np.float32))
+    exact = ci + ai @ bi.T
+    assert np.array_equal(d64, exact.astype(np.float64))
+    assert np.array_equal(d32, exact.astype(np.float32))
+
+
+def test_acc_zero_operand_returns_c(oracle_mod):
+    # A = 0 (code 0x00): D = C bit for bit (C without negative zeros, which
+    # -0 + +0 would turn positive), including subnormal and huge values
+    rng = np.random.default_rng(16)
+    M, N, K = 8, 32, 128
+    c = (rng.standard_normal((M, N)) * np.exp2(rng.integers(-140, 120, (M, N)))).astype(np.float32)
+    c[c == 0] = 1.0
+    p = gi.dense_problem(M, N, K, seed_b=17)
+    d64, d32 = oracle_mod.gemm_nt_acc(np.zeros((M, K), np.uint8), p["sA"], p["B"], p["sB"], c)
+    assert np.array_equal(d32.view(np.uint32), c.view(np.uint32))
+
+
+def test_acc_equals_c_plus_dequantised_matmul(oracle_mod):
+    p = gi.dense_problem(50, 272, 384, seed_a=18, seed_b=19)
+    c = np.random.default_rng(20).standard_normal((50, 272)).astype(np.float32) * 30
+    d64, d32 = oracle_mod.gemm_nt_acc(p["A"], p["sA"], p["B"], p["sB"], c)
+    a = _dequant(p["A"], p["sA"], 1)
+    b = _dequant(p["B"], p["sB"], BLOCK)
+    ref = c.astype(np.float64) + a @ b.T
+    bound = np.abs(c.astype(np.float64)) + np.abs(a) @ np.abs(b).T
+    assert np.all(np.abs(d64 - ref) <= 1e-12 * bound + 1e-300)
+    # one rounding from double to float32 (numpy's conversion, to nearest even)
+    assert np.array_equal(d32.view(np.uint32), d64.astype(np.float32).view(np.uint32))
+    r = np.random.default_rng(0).integers(0, 50, 300)
+    q = np.random.default_rng(1).integers(0, 272, 300)
+    s64, s32 = oracle_mod.gemm_nt_acc_sampled(p["A"], p["sA"], p["B"], p["sB"], c, r, q)
+    assert np.array_equal(s64, d64[r, q]) and np.array_equal(s32, d32[r, q])
+
+
 # ----------------------------------------------------------------- grouped
 
 SENTINEL = 0x7FC1  # a NaN pattern nobody computes
