@@ -92,6 +92,20 @@ dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B,
                            cudaStream_t stream);
 
 /*
+ * Dense NT GEMM with an accumulator: D = C + A @ B^T, the "D = C + A @ B"
+ * form of the pages (hada.io page, section "Giao dien GEMM va rang buoc
+ * layout": fp8_gemm_nt computes D = C + A @ B.T).  The pages give C no
+ * type; here C and D are fp32 [M][N], row-major, 16-byte aligned, and C may
+ * be D itself (in-place accumulation, D += A @ B^T).  A, sA, B, sB and the
+ * layout rules are those of dg_fp8_gemm_nt; the fp32 promotion accumulator
+ * of each output is added to C in fp32.  C == NULL returns
+ * DG_ERR_INVALID_ARG.  M == 0 is a no-op returning DG_OK.
+ */
+dg_status_t dg_fp8_gemm_nt_acc(const void *A, const float *sA, const void *B,
+                               const float *sB, const float *C, float *D, int M, int N,
+                               int K, cudaStream_t stream);
+
+/*
  * Contiguous-layout grouped GEMM (MoE, grouping along M; N and K shared).
  *   A         : [M_total][K]     e4m3; the rows of all groups concatenated
  *   sA        : [K/128][M_pad]   fp32, M_pad = dg_get_tma_aligned_size(M_total, 4)

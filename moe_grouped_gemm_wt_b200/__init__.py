@@ -39,6 +39,7 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SIGNATURES = {
     "dg_fp8_gemm_nt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "dg_fp8_gemm_nt_acc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_grouped_gemm_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_fp8_grouped_gemm_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
@@ -228,6 +229,29 @@ def dg_fp8_gemm_nt(A, sA, B, sB, D, stream=None) -> None:
         raise ValueError("D must be [M, N]")
     st = load_library().dg_fp8_gemm_nt(pa, psa, pb, psb, pd, M, N, K, _stream_handle(stream, A.device))
     _check("dg_fp8_gemm_nt", st)
+
+
+def dg_fp8_gemm_nt_acc(A, sA, B, sB, C, D, stream=None) -> None:
+    """D = C + A @ B^T with float32 C and D of shape [M, N] (C may be D)."""
+    pa = _dev(A, "A", _FP8, 2)
+    M, K = A.shape
+    N = B.shape[0] if B.dim() == 2 else -1
+    pb = _dev(B, "B", _FP8, 2)
+    if B.shape[1] != K:
+        raise ValueError("B must be [N, K]")
+    psa = _dev(sA, "sA", _F32, 2)
+    if tuple(sA.shape) != (K // 128, get_tma_aligned_size(M, 4)):
+        raise ValueError(f"sA must be [K/128, M_pad] = {(K // 128, get_tma_aligned_size(M, 4))}")
+    psb = _dev(sB, "sB", _F32, 2)
+    if tuple(sB.shape) != ((N + 127) // 128, K // 128):
+        raise ValueError("sB must be [ceil(N/128), K/128]")
+    pc = _dev(C, "C", _F32, 2)
+    pd = _dev(D, "D", _F32, 2)
+    if tuple(C.shape) != (M, N) or tuple(D.shape) != (M, N):
+        raise ValueError("C and D must be [M, N]")
+    st = load_library().dg_fp8_gemm_nt_acc(pa, psa, pb, psb, pc, pd, M, N, K,
+                                           _stream_handle(stream, A.device))
+    _check("dg_fp8_gemm_nt_acc", st)
 
 
 def dg_fp8_grouped_gemm_contiguous(A, sA, B, sB, D, m_indices, stream=None) -> None:

@@ -589,6 +589,49 @@ dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B, const 
                                 sms, stream);
 }
 
+dg_status_t dg_fp8_gemm_nt_acc(const void *A, const float *sA, const void *B, const float *sB,
+                               const float *C, float *D, int M, int N, int K, cudaStream_t stream)
+{
+    if (M < 0 || !C)
+        return DG_ERR_INVALID_ARG;
+    dg_status_t st = check_common(A, sA, B, sB, D, N, K);
+    if (st != DG_OK)
+        return st;
+    if (!aligned(C, 16))
+        return DG_ERR_ALIGNMENT;
+    if (M == 0)
+        return DG_OK;
+    const int dev = current_device();
+    const int sms = effective_sms(dev);
+    if (sms <= 0)
+        return DG_ERR_CUDA;
+    GemmParams p{};
+    p.sA = sA;
+    p.sB = sB;
+    // The bf16 output pointer only shapes the (unused) store tensor maps;
+    // the kernels write D through D32.
+    p.D = reinterpret_cast<__nv_bfloat16 *>(D);
+    p.C = C;
+    p.D32 = D;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = 1;
+    p.sa_ld = dg_get_tma_aligned_size(M, 4);
+    p.num_kb = K / 128;
+    p.nbn = (N + 127) / 128;
+    p.num_mb = (M + 127) / 128;
+    p.raster = choose_raster(p.num_mb);
+    p.timeout_ns = g_timeout_ns.load();
+    p.stall_injection = g_stall_injection.load();
+    const Plan plan = choose_plan(p.num_mb, (M + 255) / 256, N, p.num_kb, sms, true);
+    if (print_configs())
+        std::fprintf(stderr, "[dg] dense accumulate M=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d ksplit=%d sms=%d\n",
+                     M, N, K, plan.c.pair ? 256 : 128, plan.c.bn, plan.c.stages, plan.c.ks, plan.ksplit, sms);
+    return dispatch<dg::kDense>(plan, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), p,
+                                sms, stream);
+}
+
 dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const void *B,
                                            const float *sB, void *D, const int32_t *m_indices,
                                            int M_total, int N, int K, int num_groups,

@@ -92,7 +92,28 @@ struct GemmParams {
     float *ws;                // K split: fp32 partials [tile][split][BN/4][128][4]
     int stall_injection;      // test hook: CTA 0's producer issues nothing
     unsigned long long timeout_ns;
+    // Dense accumulate form D = C + A.B^T: when D32 is set the output is
+    // fp32 D32[M][N] = C[M][N] + acc (C may be D32 itself) instead of bf16 D.
+    const float *C;
+    float *D32;
 };
+
+// Row segment of the accumulate form: drow[c] = crow[c] + acc[c] for the
+// 4-float groups of this thread's row that lie inside N (read before write,
+// so crow == drow is fine).
+template <int COLS>
+__device__ __forceinline__ void store_row_acc_f32(const float *crow, float *drow, const float *acc, int col0,
+                                                  int N)
+{
+#pragma unroll
+    for (int c = 0; c < COLS; c += 4) {
+        if (col0 + c < N) {
+            const float4 cv = *reinterpret_cast<const float4 *>(crow + c);
+            *reinterpret_cast<float4 *>(drow + c) =
+                make_float4(cv.x + acc[c], cv.y + acc[c + 1], cv.z + acc[c + 2], cv.w + acc[c + 3]);
+        }
+    }
+}
 
 constexpr int kBM = 128;
 constexpr int kBK = 128;
@@ -664,6 +685,16 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                 ok = false;
                 break;
             }
+            if constexpr (LAYOUT == kDense) {
+                if (p.D32) {
+                    // accumulate form: fp32 C + acc, row by row
+                    if (row_ok)
+                        store_row_acc_f32<BN_WG>(p.C + static_cast<size_t>(m_local) * p.N + col0,
+                                                 p.D32 + static_cast<size_t>(m_local) * p.N + col0, acc, col0,
+                                                 p.N);
+                    continue;
+                }
+            }
             const bool tile_rows_ok = named_barrier_and(
                 1 + wg, 128, LAYOUT == kDense ? (tc.mb * kBM < p.M) : row_ok);
             if (tile_rows_ok) {
@@ -752,7 +783,13 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                 }
                 const int grow = tc.mb * kBM + r;
                 const int gcol = tc.nb * BN + c4 * 4;
-                if (grow < p.M && gcol < p.N) {
+                if (grow < p.M && gcol < p.N && p.D32) {
+                    // accumulate form: fp32 C + sum
+                    const size_t off = static_cast<size_t>(grow) * p.N + gcol;
+                    const float4 cv = *reinterpret_cast<const float4 *>(p.C + off);
+                    *reinterpret_cast<float4 *>(p.D32 + off) =
+                        make_float4(cv.x + sum.x, cv.y + sum.y, cv.z + sum.z, cv.w + sum.w);
+                } else if (grow < p.M && gcol < p.N) {
                     __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
                     __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
                     uint2 u;

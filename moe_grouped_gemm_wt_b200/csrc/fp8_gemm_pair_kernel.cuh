@@ -552,6 +552,16 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG>::THREADS, 1)
                 ok = false;
                 break;
             }
+            if constexpr (LAYOUT == kDense) {
+                if (p.D32) {
+                    // accumulate form: fp32 C + acc, row by row
+                    if (row_ok)
+                        store_row_acc_f32<BN_WG>(p.C + static_cast<size_t>(m_local) * p.N + col0,
+                                                 p.D32 + static_cast<size_t>(m_local) * p.N + col0, acc, col0,
+                                                 p.N);
+                    continue;
+                }
+            }
             const bool tile_rows_ok = named_barrier_and(
                 1 + wg, 128, LAYOUT == kDense ? (m_half < p.M) : row_ok);
             if (tile_rows_ok) {

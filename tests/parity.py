@@ -51,6 +51,24 @@ def assert_close(got_bits: np.ndarray, ref_bits: np.ndarray, what: str = ""):
     return cd
 
 
+def assert_close_f32(got: np.ndarray, ref: np.ndarray, what: str = ""):
+    """The same tolerance for fp32 outputs (the accumulate form)."""
+    got = got.astype(np.float64)
+    ref = ref.astype(np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    bound = REL_TOL * (np.abs(ref) + ABS_FLOOR)
+    bad = err > bound
+    if bad.any():
+        i = np.argmax(err / bound)
+        raise AssertionError(
+            f"{what}: {int(bad.sum())} of {bad.size} elements beyond tolerance; worst at flat "
+            f"{int(i)}: got {got.ravel()[i]!r} oracle {ref.ravel()[i]!r}")
+    cd = calc_diff(got, ref)
+    assert cd <= CALC_DIFF_MAX, f"{what}: calc_diff {cd:.3e} > {CALC_DIFF_MAX}"
+    return cd
+
+
 def dev_dense(p):
     """Dense problem -> device tensors in the library layout (+ D prefilled)."""
     dev = torch.device("cuda")
