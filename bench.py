@@ -220,6 +220,34 @@ def whole_job_value(flop_per_rank, world, ms):
     return flop_per_rank * world / (ms * 1e-3) / 1e12
 
 
+def shard_experts(p, rank, world):
+    """Expert parallelism for the grouped workloads: rank r keeps experts
+    [r*G/world, (r+1)*G/world) -- their rows of A and sA (contiguous: the
+    groups' segments, each with the padding rows that follow it; masked:
+    whole groups), their B, sB and metadata, with group indices renumbered
+    from 0.  No exchange is needed: every expert's output rows live on the
+    rank that computes them."""
+    G = p["G"]
+    g0, g1 = rank * G // world, (rank + 1) * G // world
+    q = dict(p)
+    q["G"] = g1 - g0
+    q["B"], q["sB"] = p["B"][g0:g1], p["sB"][g0:g1]
+    if p["kind"] == "masked":
+        for k in ("A", "sA", "masked_m"):
+            q[k] = p[k][g0:g1]
+        return q
+    mi = np.asarray(p["m_indices"])
+    # owner of each row: its group, or for a padding row the group before it
+    owner = np.maximum.accumulate(np.where(mi >= 0, mi, -1))
+    owner[owner < 0] = 0
+    rows = np.flatnonzero((owner >= g0) & (owner < g1))
+    lo, hi = (int(rows[0]), int(rows[-1]) + 1) if rows.size else (0, 0)
+    q["A"], q["sA"] = p["A"][lo:hi], p["sA"][lo:hi]
+    q["m_indices"] = np.where(mi[lo:hi] >= 0, mi[lo:hi] - g0, -1).astype(np.int32)
+    q["M"] = hi - lo
+    return q
+
+
 def workload_label(p, name):
     if p["kind"] == "dense":
         return f"{name} M={p['M']} N={p['N']} K={p['K']}"
@@ -364,6 +392,15 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     p = gi.make_workload(args.workload)
+    # Grouped workloads on several ranks: expert parallel, the fixed problem
+    # split by expert (strong scaling); dense workloads: one replica per rank
+    # (weak scaling).
+    expert_parallel = world > 1 and p["kind"] != "dense"
+    flop_job = workload_cost(p)[0] if expert_parallel else None
+    if expert_parallel:
+        if world > p["G"]:
+            raise SystemExit(f"expert parallel: {world} ranks for {p['G']} experts")
+        p = shard_experts(p, rank, world)
     d = to_device(p, torch, dev)
     flop, byts, _ = workload_cost(p)
 
@@ -382,8 +419,9 @@ def run_ours(args):
     shapes = {}
     if not args.no_shapes:
         for name in gi.WORKLOADS:
-            q = p if name == args.workload else gi.make_workload(name)
-            dq = d if name == args.workload else to_device(q, torch, dev)
+            same = name == args.workload and not expert_parallel  # a shard is not the shape
+            q = p if same else gi.make_workload(name)
+            dq = d if same else to_device(q, torch, dev)
             tq = time_kernel(torch, dg, q, dq, max(10, min(args.steps, 30)), 3, flush)
             mq = statistics.median(tq)
             fq, bq, rows = workload_cost(q)
@@ -394,14 +432,14 @@ def run_ours(args):
                 "frac_of_roofline": t_roof / (mq * 1e-3),
                 "valid_rows": rows,
             }
-            if name != args.workload:
+            if not same:
                 del dq
                 torch.cuda.empty_cache()
     clocks = sampler.stop()
 
     e2e_ms, h2d, d2h = time_e2e(torch, dg, p, max(10, min(args.steps, 50)), 3, dev)
 
-    value = whole_job_value(flop, world, ms)
+    value = flop_job / (ms * 1e-3) / 1e12 if expert_parallel else whole_job_value(flop, world, ms)
     bound, t_roof, fp8_peak = roofline(flop, byts, pk)
     if bound == "hbm":
         achieved = byts / (ms * 1e-3) / 1e9
@@ -428,12 +466,13 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8_e4m3 (fp32 promotion, bf16 out)",
+        "higher_is_better": True, "scaling": "strong" if expert_parallel else "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 promotion, bf16 out)",
         "data": "synthetic (seeded N(0,1) quantised to e4m3 with 1x128 / 128x128 fp32 scales)",
         "config": {"workload": workload_label(p, args.workload),
                    "l2": "flushed before every timed launch (512 MiB write)",
-                   "parallelism": f"replicas x{world}",
+                   "parallelism": (f"expert parallel x{world} (this rank: {p['G']} experts)"
+                                   if expert_parallel else f"replicas x{world}"),
                    "tile": tile_label(dg, p)},
         "roofline": roof,
         "frac_of_roofline": t_roof / (ms * 1e-3),

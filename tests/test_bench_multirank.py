@@ -58,3 +58,51 @@ def test_reference_arm_is_silent_on_other_ranks(capsys, monkeypatch):
     monkeypatch.setenv("RANK", "1")
     assert bench.run_reference(Args()) == 0
     assert capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("world", [2, 3, 8])
+def test_expert_shards_partition_the_grouped_problems(oracle_mod, world):
+    """Each rank's shard holds whole experts (renumbered from 0); together
+    the shards hold every expert once, and each shard's oracle result equals
+    the rows of the whole problem's result that belong to its experts."""
+    import sys
+    import numpy as np
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    import dg_inputs as gi
+
+    SENT = 0x7FC1
+    # contiguous: uneven groups, an empty group, padding rows
+    p = gi.contiguous_problem([100, 300, 0, 37, 128, 5, 260, 64], 144, 256, seed_a=91, seed_b=92)
+    full = oracle_mod.grouped_contiguous(p["A"], p["sA"], p["B"], p["sB"], p["m_indices"],
+                                         np.full((p["M"], 144), SENT, np.uint16))[1]
+    seen_rows = 0
+    total_flop = 0.0
+    lo = 0
+    for r in range(world):
+        q = bench.shard_experts(p, r, world)
+        g0 = r * p["G"] // world
+        assert q["G"] == (r + 1) * p["G"] // world - g0
+        assert q["M"] % 128 == 0 and np.all(q["m_indices"] < q["G"])
+        part = oracle_mod.grouped_contiguous(q["A"], q["sA"], q["B"], q["sB"], q["m_indices"],
+                                             np.full((q["M"], 144), SENT, np.uint16))[1]
+        assert np.array_equal(part, full[lo:lo + q["M"]])
+        lo += q["M"]
+        seen_rows += q["M"]
+        total_flop += bench.workload_cost(q)[0]
+    assert seen_rows == p["M"]
+    assert total_flop == bench.workload_cost(p)[0]
+
+    # masked: whole groups
+    pm = gi.masked_problem(5, 200, 144, 256, masked_m=[0, 200, 77, 150, 3], seed_a=93, seed_b=94)
+    fullm = oracle_mod.grouped_masked(pm["A"], pm["sA"], pm["B"], pm["sB"], pm["masked_m"],
+                                      np.full((5, 200, 144), SENT, np.uint16))[1]
+    got = []
+    for r in range(world):
+        q = bench.shard_experts(pm, r, world)
+        if q["G"] == 0:
+            continue  # more ranks than experts: this rank has none
+        got.append(oracle_mod.grouped_masked(q["A"], q["sA"], q["B"], q["sB"], q["masked_m"],
+                                             np.full((q["G"], 200, 144), SENT, np.uint16))[1])
+    assert np.array_equal(np.concatenate(got), fullm)
