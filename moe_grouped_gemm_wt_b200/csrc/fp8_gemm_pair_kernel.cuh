@@ -140,7 +140,9 @@ struct PairConfig {
     static constexpr int KS = KS_;
     static constexpr int NUM_WG = NWG_;     // promotion warpgroups
     static constexpr int BN_WG = BN / NUM_WG;
-    static constexpr int RMAX = BN_WG <= 64 ? BN_WG : 32;
+    // TMEM load rounds: the whole partial when it fits beside the
+    // accumulator, else halves of up to 40 columns, else rounds of 32.
+    static constexpr int RMAX = BN_WG <= 64 ? BN_WG : (BN_WG <= 80 ? BN_WG / 2 : 32);
     static constexpr int NUM_PROMO_WARPS = 4 * NUM_WG;
     static constexpr int PRODUCER_A_WARP = NUM_PROMO_WARPS;
     static constexpr int PRODUCER_B_WARP = NUM_PROMO_WARPS + 1;
