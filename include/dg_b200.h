@@ -92,6 +92,31 @@ dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B,
                            cudaStream_t stream);
 
 /*
+ * The other three operand layouts of the dense GEMM (hada.io page, section
+ * "Giao dien GEMM va rang buoc layout": the SM100 implementation supports
+ * the NT, TN, NN and TT memory layouts).  Read as D = op(A) @ op(B) with
+ * row-major storage, the letter n for an operand stored in its logical
+ * shape (A as [M][K], B as [K][N]) and t for one stored transposed (A as
+ * [K][M], B as [N][K]); dg_fp8_gemm_nt is the NT case:
+ *   nn : A [M][K] (K-major),  B [K][N] (N-major)
+ *   tn : A [K][M] (M-major),  B [K][N] (N-major)
+ *   tt : A [K][M] (M-major),  B [N][K] (K-major)
+ * sA, sB and D are as in dg_fp8_gemm_nt (sA [K/128][M_pad], sB
+ * [ceil(N/128)][K/128], D [M][N] bf16).  An M-major A needs M % 16 == 0
+ * (DG_ERR_UNSUPPORTED otherwise).  These layouts run on one-CTA tiles; an
+ * N-major B uses 128- or 256-column tiles and no K split.
+ */
+dg_status_t dg_fp8_gemm_nn(const void *A, const float *sA, const void *B,
+                           const float *sB, void *D, int M, int N, int K,
+                           cudaStream_t stream);
+dg_status_t dg_fp8_gemm_tn(const void *A, const float *sA, const void *B,
+                           const float *sB, void *D, int M, int N, int K,
+                           cudaStream_t stream);
+dg_status_t dg_fp8_gemm_tt(const void *A, const float *sA, const void *B,
+                           const float *sB, void *D, int M, int N, int K,
+                           cudaStream_t stream);
+
+/*
  * Dense NT GEMM with an accumulator: D = C + A @ B^T, the "D = C + A @ B"
  * form of the pages (hada.io page, section "Giao dien GEMM va rang buoc
  * layout": fp8_gemm_nt computes D = C + A @ B.T).  The pages give C no

@@ -40,6 +40,9 @@ _I = ctypes.c_int
 _SIGNATURES = {
     "dg_fp8_gemm_nt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_acc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "dg_fp8_gemm_nn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "dg_fp8_gemm_tn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "dg_fp8_gemm_tt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_grouped_gemm_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_fp8_grouped_gemm_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
@@ -229,6 +232,44 @@ def dg_fp8_gemm_nt(A, sA, B, sB, D, stream=None) -> None:
         raise ValueError("D must be [M, N]")
     st = load_library().dg_fp8_gemm_nt(pa, psa, pb, psb, pd, M, N, K, _stream_handle(stream, A.device))
     _check("dg_fp8_gemm_nt", st)
+
+
+def _dense_layout(name, a_t, b_n, A, sA, B, sB, D, stream):
+    pa = _dev(A, "A", _FP8, 2)
+    pb = _dev(B, "B", _FP8, 2)
+    if a_t:
+        K, M = A.shape
+    else:
+        M, K = A.shape
+    N = B.shape[1] if b_n else B.shape[0]
+    if (B.shape[0] if b_n else B.shape[1]) != K:
+        raise ValueError(f"{name}: B must be {'[K, N]' if b_n else '[N, K]'} with K = {K}")
+    psa = _dev(sA, "sA", _F32, 2)
+    if tuple(sA.shape) != (K // 128, get_tma_aligned_size(M, 4)):
+        raise ValueError(f"sA must be [K/128, M_pad] = {(K // 128, get_tma_aligned_size(M, 4))}")
+    psb = _dev(sB, "sB", _F32, 2)
+    if tuple(sB.shape) != ((N + 127) // 128, K // 128):
+        raise ValueError("sB must be [ceil(N/128), K/128]")
+    pd = _dev(D, "D", _BF16, 2)
+    if tuple(D.shape) != (M, N):
+        raise ValueError("D must be [M, N]")
+    st = getattr(load_library(), name)(pa, psa, pb, psb, pd, M, N, K, _stream_handle(stream, A.device))
+    _check(name, st)
+
+
+def dg_fp8_gemm_nn(A, sA, B, sB, D, stream=None) -> None:
+    """D = A @ B with A [M, K] and B [K, N] (N-major)."""
+    _dense_layout("dg_fp8_gemm_nn", False, True, A, sA, B, sB, D, stream)
+
+
+def dg_fp8_gemm_tn(A, sA, B, sB, D, stream=None) -> None:
+    """D = A^T @ B with A stored [K, M] (M-major) and B [K, N] (N-major)."""
+    _dense_layout("dg_fp8_gemm_tn", True, True, A, sA, B, sB, D, stream)
+
+
+def dg_fp8_gemm_tt(A, sA, B, sB, D, stream=None) -> None:
+    """D = A^T @ B^T with A stored [K, M] (M-major) and B stored [N, K]."""
+    _dense_layout("dg_fp8_gemm_tt", True, False, A, sA, B, sB, D, stream)
 
 
 def dg_fp8_gemm_nt_acc(A, sA, B, sB, C, D, stream=None) -> None:

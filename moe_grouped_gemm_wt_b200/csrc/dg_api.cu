@@ -71,6 +71,22 @@ bool make_tmap_operand(CUtensorMap *map, const void *base, uint64_t K, uint64_t 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// An MN-major e4m3 operand stored [K][inner] (inner = M for A, N for B):
+// 2-D boxes of 128 inner bytes by box_k K rows, 128-byte swizzled.
+bool make_tmap_mn(CUtensorMap *map, const void *base, uint64_t inner, uint64_t K, uint32_t box_k)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {inner, K};
+    cuuint64_t strides[1] = {inner};
+    cuuint32_t box[2] = {128, box_k};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 matrix [rows][inner] (the output), box [box_rows][box_inner].
 bool make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                     uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle)
@@ -223,13 +239,32 @@ int max_active_clusters(const TileChoice &c, int S);
 // range of each tile may be split over a cluster of 2..16 CTAs.  Pair tiles
 // (256 rows on two SMs) are taken only by problems with at least one full
 // wave of them.  m_blocks counts 128-row blocks, pair_rows 256-row ones.
-Plan choose_plan(int64_t m_blocks, int64_t pair_rows, int N, int num_kb, int sms, bool allow_split)
+// Operand layouts restrict the choice: MN-major operands run on one-CTA
+// tiles only (kNoPair), and an MN-major B needs whole 128-column boxes
+// (kWholeBoxes: BN % 128 == 0, no K split).
+constexpr int kNoPair = 1;
+constexpr int kWholeBoxes = 2;
+
+Plan choose_plan(int64_t m_blocks, int64_t pair_rows, int N, int num_kb, int sms, bool allow_split,
+                 int limits = 0)
 {
     Plan best{kTileChoices[0], 1};
     double best_cost = 1e300;
+    if (limits & kWholeBoxes) {
+        allow_split = false;
+        for (const TileChoice &c : kTileChoices)
+            if (!c.pair && !c.split && c.bn % 128 == 0) {
+                best = Plan{c, 1};
+                break;
+            }
+    }
     for (const TileChoice &c : kTileChoices) {
         const bool forced = forced_block_n() > 0;
         if (forced && c.bn != forced_block_n())
+            continue;
+        if ((limits & (kNoPair | kWholeBoxes)) && c.pair)
+            continue;
+        if ((limits & kWholeBoxes) && c.bn % 128 != 0)
             continue;
         if (forced_pair() >= 0 && c.pair != forced_pair())
             continue;
@@ -282,14 +317,17 @@ int choose_raster(int num_mb)
     return num_mb < 16 ? (num_mb > 0 ? num_mb : 1) : 16;
 }
 
-template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT>
+template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false>
 dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
                           const GemmParams &p, int grid, cudaStream_t stream)
 {
     using Cfg = KernelConfig<BN, STAGES, KS, SPLIT>;
     CUtensorMap ta, tb;
-    if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
-        !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, BN, KS))
+    const bool ok_a = A_MN ? make_tmap_mn(&ta, A, a_rows, static_cast<uint64_t>(p.K), KS * dg::kBK)
+                           : make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS);
+    const bool ok_b = B_MN ? make_tmap_mn(&tb, B, b_rows, static_cast<uint64_t>(p.K), KS * dg::kBK)
+                           : make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, BN, KS);
+    if (!ok_a || !ok_b)
         return DG_ERR_CUDA;
     const uint64_t d_rows = a_rows;
     // output boxes of 32 rows: 64 columns with 128-byte swizzle, and the
@@ -305,7 +343,7 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
     } else {
         tdrem = td64;
     }
-    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT, SPLIT>;
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT, SPLIT, A_MN, B_MN>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices)
@@ -472,12 +510,14 @@ int max_active_clusters(const TileChoice &c, int S)
     return n < 0 ? 0 : (n < cap ? n : cap);
 }
 
-template <int LAYOUT>
+template <int LAYOUT, bool A_MN = false, bool B_MN = false>
 dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const void *B,
                      uint64_t b_rows, GemmParams p, int sms, cudaStream_t stream)
 {
     const TileChoice &c = plan.c;
     p.num_nb = (p.N + c.bn - 1) / c.bn;
+    if ((A_MN || B_MN) && c.pair)
+        return DG_ERR_UNSUPPORTED;  // the planner keeps MN-major operands on one-CTA tiles
     if (c.pair) {
         // the pair scheduler counts 256-row pair rows
         p.num_mb = (p.num_mb + 1) / 2;
@@ -516,17 +556,21 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
         grid = static_cast<int>(tiles < sms ? tiles : sms);
     if (grid <= 0)
         return DG_OK;
-#define DG_TILE_CASE(BN_, ST_, KS_)                                                         \
-    if (c.bn == BN_ && c.stages == ST_ && c.ks == KS_ && !c.split)                           \
-        return launch_kernel<BN_, ST_, KS_, LAYOUT, false>(A, a_rows, B, b_rows, p, grid, stream);
+#define DG_TILE_CASE(BN_, ST_, KS_)                                                          \
+    if constexpr (!B_MN || BN_ % 128 == 0) {                                                  \
+        if (c.bn == BN_ && c.stages == ST_ && c.ks == KS_ && !c.split)                        \
+            return launch_kernel<BN_, ST_, KS_, LAYOUT, false, A_MN, B_MN>(A, a_rows, B, b_rows, p, \
+                                                                           grid, stream);     \
+    }
     DG_TILE_CASE(112, 3, 2)
     DG_TILE_CASE(128, 5, 1)
     DG_TILE_CASE(224, 2, 2)
     DG_TILE_CASE(256, 3, 1)
 #undef DG_TILE_CASE
-    if constexpr (LAYOUT == dg::kDense) {
+    if constexpr (LAYOUT == dg::kDense && !B_MN) {
         if (c.bn == 144 && c.stages == 3 && c.ks == 2 && c.split)
-            return launch_kernel<144, 3, 2, LAYOUT, true>(A, a_rows, B, b_rows, p, grid, stream);
+            return launch_kernel<144, 3, 2, LAYOUT, true, A_MN, false>(A, a_rows, B, b_rows, p, grid,
+                                                                       stream);
     }
     return DG_ERR_UNSUPPORTED;
 }
@@ -546,20 +590,18 @@ dg_status_t check_common(const void *A, const float *sA, const void *B, const fl
     return DG_OK;
 }
 
-}  // namespace
-
-// =================================================================== C ABI
-
-extern "C" {
-
-dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B, const float *sB,
-                           void *D, int M, int N, int K, cudaStream_t stream)
+// The dense GEMM in any of the four operand layouts: A K-major ([M][K]) or
+// M-major ([K][M], a_mn), B K-major ([N][K]) or N-major ([K][N], b_mn).
+dg_status_t dense_gemm(const void *A, const float *sA, const void *B, const float *sB, void *D,
+                       int M, int N, int K, bool a_mn, bool b_mn, cudaStream_t stream)
 {
     if (M < 0)
         return DG_ERR_INVALID_ARG;
     dg_status_t st = check_common(A, sA, B, sB, D, N, K);
     if (st != DG_OK)
         return st;
+    if (a_mn && M % 16 != 0)
+        return DG_ERR_UNSUPPORTED;  // rows of an M-major A must be whole 16-byte units
     if (M == 0)
         return DG_OK;
     const int dev = current_device();
@@ -581,12 +623,50 @@ dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B, const 
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
     p.stall_injection = g_stall_injection.load();
-    const Plan plan = choose_plan(p.num_mb, (M + 255) / 256, N, p.num_kb, sms, true);
+    const int limits = (a_mn || b_mn ? kNoPair : 0) | (b_mn ? kWholeBoxes : 0);
+    const Plan plan = choose_plan(p.num_mb, (M + 255) / 256, N, p.num_kb, sms, true, limits);
     if (print_configs())
-        std::fprintf(stderr, "[dg] dense M=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d ksplit=%d sms=%d\n",
-                     M, N, K, plan.c.pair ? 256 : 128, plan.c.bn, plan.c.stages, plan.c.ks, plan.ksplit, sms);
-    return dispatch<dg::kDense>(plan, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), p,
-                                sms, stream);
+        std::fprintf(stderr, "[dg] dense %s%s M=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d ksplit=%d sms=%d\n",
+                     a_mn ? "t" : "n", b_mn ? "n" : "t", M, N, K, plan.c.pair ? 256 : 128, plan.c.bn,
+                     plan.c.stages, plan.c.ks, plan.ksplit, sms);
+    const uint64_t am = static_cast<uint64_t>(M), bn = static_cast<uint64_t>(N);
+    if (a_mn && b_mn)
+        return dispatch<dg::kDense, true, true>(plan, A, am, B, bn, p, sms, stream);
+    if (a_mn)
+        return dispatch<dg::kDense, true, false>(plan, A, am, B, bn, p, sms, stream);
+    if (b_mn)
+        return dispatch<dg::kDense, false, true>(plan, A, am, B, bn, p, sms, stream);
+    return dispatch<dg::kDense>(plan, A, am, B, bn, p, sms, stream);
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+
+extern "C" {
+
+dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B, const float *sB,
+                           void *D, int M, int N, int K, cudaStream_t stream)
+{
+    return dense_gemm(A, sA, B, sB, D, M, N, K, false, false, stream);
+}
+
+dg_status_t dg_fp8_gemm_nn(const void *A, const float *sA, const void *B, const float *sB,
+                           void *D, int M, int N, int K, cudaStream_t stream)
+{
+    return dense_gemm(A, sA, B, sB, D, M, N, K, false, true, stream);
+}
+
+dg_status_t dg_fp8_gemm_tn(const void *A, const float *sA, const void *B, const float *sB,
+                           void *D, int M, int N, int K, cudaStream_t stream)
+{
+    return dense_gemm(A, sA, B, sB, D, M, N, K, true, true, stream);
+}
+
+dg_status_t dg_fp8_gemm_tt(const void *A, const float *sA, const void *B, const float *sB,
+                           void *D, int M, int N, int K, cudaStream_t stream)
+{
+    return dense_gemm(A, sA, B, sB, D, M, N, K, true, false, stream);
 }
 
 dg_status_t dg_fp8_gemm_nt_acc(const void *A, const float *sA, const void *B, const float *sB,

@@ -339,7 +339,12 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float *v)
 
 // ------------------------------------------------------------------ kernel
 
-template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT>
+// A_MN / B_MN: the operand is stored MN-major (A as [K][M], B as [K][N],
+// the "t" layouts of the A operand and the "n" layouts of the B operand; dense
+// only).  Its stage tile is then loaded as 2-D TMA boxes of 128 M (or N)
+// bytes by 128*KS K rows (B: one box per 128 columns, BN % 128 == 0) and
+// described to the MMA as an MN-major 128-byte-swizzled operand.
+template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false>
 __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
@@ -348,6 +353,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
 {
     using Cfg = KernelConfig<BN, STAGES, KS, SPLIT>;
     static_assert(!SPLIT || LAYOUT == kDense, "K split is implemented for the dense layout");
+    static_assert((!A_MN && !B_MN) || LAYOUT == kDense, "MN-major operands are implemented for the dense layout");
+    static_assert(!B_MN || BN % 128 == 0, "an MN-major B tile is whole 128-column boxes");
     constexpr int BN_WG = Cfg::BN_WG;
     constexpr int RMAX = Cfg::RMAX;
     constexpr int NBUF = Cfg::NBUF;
@@ -444,10 +451,22 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                 const uint32_t fb = smem_addr(full_bar + stage);
                 if (elect_one()) {
                     mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
-                    tma_load_3d(smem_addr(a_tiles + stage * KS * Cfg::A_BYTES), &tmap_a, fb, 0,
-                                a_row, kb0);
-                    tma_load_3d(smem_addr(b_tiles + stage * KS * Cfg::B_BYTES), &tmap_b, fb, 0,
-                                b_row, kb0);
+                    if constexpr (A_MN)
+                        tma_load_2d(smem_addr(a_tiles + stage * KS * Cfg::A_BYTES), &tmap_a, fb, a_row,
+                                    kb0 * kBK);
+                    else
+                        tma_load_3d(smem_addr(a_tiles + stage * KS * Cfg::A_BYTES), &tmap_a, fb, 0,
+                                    a_row, kb0);
+                    if constexpr (B_MN) {
+                        // [BN/128 column slices][KS*128 K rows][128 bytes]
+#pragma unroll
+                        for (int c = 0; c < BN / 128; ++c)
+                            tma_load_2d(smem_addr(b_tiles + stage * KS * Cfg::B_BYTES + c * KS * kBK * 128),
+                                        &tmap_b, fb, b_row + c * 128, kb0 * kBK);
+                    } else {
+                        tma_load_3d(smem_addr(b_tiles + stage * KS * Cfg::B_BYTES), &tmap_b, fb, 0,
+                                    b_row, kb0);
+                    }
                 }
 #pragma unroll
                 for (int q = 0; q < KS; ++q) {
@@ -493,9 +512,16 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
         // every MMA issued before it has completed
         uint32_t last_bar = 0, last_parity = 0;
         bool ok = true;
-        constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BN);
-        const uint64_t a_desc0 = smem_desc_k_sw128(smem_addr(a_tiles));
-        const uint64_t b_desc0 = smem_desc_k_sw128(smem_addr(b_tiles));
+        constexpr uint32_t idesc = idesc_e4m3_f32(kBM, BN, A_MN, B_MN);
+        // K-major tiles advance 32 bytes per 32-wide K step; MN-major tiles
+        // 32 K rows of 128 bytes.  An MN-major B tile's 128-column slices
+        // lie KS*128 rows of 128 bytes apart.
+        const uint64_t a_desc0 = A_MN ? smem_desc_mn_sw128(smem_addr(a_tiles), KS * kBK * 128)
+                                      : smem_desc_k_sw128(smem_addr(a_tiles));
+        const uint64_t b_desc0 = B_MN ? smem_desc_mn_sw128(smem_addr(b_tiles), KS * kBK * 128)
+                                      : smem_desc_k_sw128(smem_addr(b_tiles));
+        constexpr uint64_t a_kstep = A_MN ? (32 * 128) >> 4 : 32 >> 4;
+        constexpr uint64_t b_kstep = B_MN ? (32 * 128) >> 4 : 32 >> 4;
         while (ok && sched.next(tc, false)) {
             const int kb_end = sched.kb_end();
             for (int kb0 = sched.kb_begin(); kb0 < kb_end; kb0 += KS) {
@@ -518,11 +544,13 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                     const uint32_t d_tmem = tmem_base + buf * Cfg::ACC_STRIDE;
                     // descriptor start address advances in 16-byte units
                     const uint64_t ad = a_desc0 + static_cast<uint64_t>(((stage * KS + q) * Cfg::A_BYTES) >> 4);
-                    const uint64_t bd = b_desc0 + static_cast<uint64_t>(((stage * KS + q) * Cfg::B_BYTES) >> 4);
+                    const uint64_t bd =
+                        b_desc0 + static_cast<uint64_t>(
+                                      (B_MN ? stage * KS * Cfg::B_BYTES + q * kBK * 128 : (stage * KS + q) * Cfg::B_BYTES) >> 4);
                     if (elect_one()) {
 #pragma unroll
                         for (int j = 0; j < kBK / 32; ++j)
-                            mma_f8f6f4(d_tmem, ad + 2 * j, bd + 2 * j, idesc, j > 0 ? 1u : 0u);
+                            mma_f8f6f4(d_tmem, ad + a_kstep * j, bd + b_kstep * j, idesc, j > 0 ? 1u : 0u);
                         mma_commit(smem_addr(tfull_bar + buf));
                     }
                     __syncwarp();

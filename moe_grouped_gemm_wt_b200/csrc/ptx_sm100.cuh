@@ -468,13 +468,29 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr)
     return d;
 }
 
-// Instruction descriptor for kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B
-// e4m3 (format 0 in bits 7-9 and 10-12), both K-major (bits 15, 16 = 0),
-// N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
+// Shared-memory matrix descriptor for an MN-major operand tile written by
+// TMA with 128-byte swizzling: each K row is 128 bytes of the M (or N)
+// dimension, 8-row atoms of 1024 bytes stacked along K (stride-dimension
+// offset 1024 B), and further 128-element slices of M/N `mn_stride` bytes
+// apart (leading-dimension offset).  Version and swizzle bits as above.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t mn_stride)
 {
-    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) |
-           (static_cast<uint32_t>(M >> 4) << 24);
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+    d |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFF) << 16;
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+// Instruction descriptor for kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B
+// e4m3 (format 0 in bits 7-9 and 10-12), A and B K-major (bits 15, 16 = 0)
+// or MN-major (= 1), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, bool a_mn = false, bool b_mn = false)
+{
+    return (1u << 4) | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 }  // namespace dg

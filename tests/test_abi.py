@@ -82,6 +82,11 @@ def test_null_and_alignment(lib):
     assert lib.dg_fp8_grouped_gemm_masked(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, -1, 256, 512, 0, None) == 1
     # empty problems are no-ops
     assert lib.dg_fp8_gemm_nt(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 512, None) == 0
+    # other layouts: an M-major A needs M % 16 == 0; the usual shape rules
+    assert lib.dg_fp8_gemm_tn(FAKE, FAKE, FAKE, FAKE, FAKE, 200, 256, 512, None) == 2
+    assert lib.dg_fp8_gemm_tt(FAKE, FAKE, FAKE, FAKE, FAKE, 200, 256, 512, None) == 2
+    assert lib.dg_fp8_gemm_nn(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 250, 512, None) == 2
+    assert lib.dg_fp8_gemm_nn(None, FAKE, FAKE, FAKE, FAKE, 128, 256, 512, None) == 1
     # accumulate form: C is required and 16-byte aligned; same shape rules
     assert lib.dg_fp8_gemm_nt_acc(FAKE, FAKE, FAKE, FAKE, None, FAKE, 128, 256, 512, None) == 1
     assert lib.dg_fp8_gemm_nt_acc(FAKE, FAKE, FAKE, FAKE, odd, FAKE, 128, 256, 512, None) == 3
