@@ -75,6 +75,19 @@ def quantize_128x128(x: np.ndarray):
     return codes, scales
 
 
+def quantize_128x1(x: np.ndarray):
+    """x: [K, C] float32 -> (codes uint8 [K, C], scales float32 [K/128, C]):
+    one scale per 128 rows of K and per column (the granularity of the
+    operands of the K-grouped weight-gradient GEMM, whose contraction runs
+    along K)."""
+    K, C = x.shape
+    assert K % BLOCK == 0
+    xb = x.reshape(K // BLOCK, BLOCK, C)
+    amax = np.abs(xb).max(axis=1)
+    scale = (np.maximum(amax, np.float32(AMAX_FLOOR)) / np.float32(E4M3_MAX)).astype(np.float32)
+    return _cast_e4m3(xb / scale[:, None, :]).reshape(K, C), scale
+
+
 def tma_aligned_size(x: int, elem_bytes: int = 4) -> int:
     """Round x up so that x * elem_bytes is a multiple of 16 bytes."""
     per = 16 // elem_bytes
@@ -109,6 +122,19 @@ def grouped_weights(G: int, N: int, K: int, seed_b: int = SEED_B):
     for g in range(G):
         B[g], sB[g] = quantize_128x128(gen.standard_normal((N, K), dtype=np.float32))
     return B, sB
+
+
+def k_grouped_problem(ks, M: int, N: int, seed_a: int = SEED_A, seed_b: int = SEED_B):
+    """K-grouped layout (MoE weight gradient): group g owns ks[g] rows (a
+    multiple of 128, possibly 0) of the shared K axis.  A [K][M] and B [K][N]
+    are stored MN-major and scaled per 128 rows of K and per column."""
+    assert all(k % BLOCK == 0 and k >= 0 for k in ks)
+    K = int(sum(ks))
+    k_offsets = np.concatenate([[0], np.cumsum(ks)]).astype(np.int32)
+    a, sa = quantize_128x1(standard_normal(seed_a, (K, M)))
+    b, sb = quantize_128x1(standard_normal(seed_b, (K, N)))
+    return dict(kind="k_grouped", A=a, sA=sa, B=b, sB=sb, k_offsets=k_offsets,
+                M=M, N=N, K=K, G=len(ks))
 
 
 def contiguous_problem(rows_per_group, N: int, K: int, seed_a: int = SEED_A,

@@ -17,6 +17,9 @@ Parity status of each function (what pins it is listed in the tests):
                                 (exact with unit scales, 1e-12 with scales),
                                 integer inputs, identity/zero, power-of-two
                                 invariance, brute-force loops on tiny cases
+  k_grouped_tn                  pinned: each group equals the float64 matmul
+                                of its dequantised slices (1e-12), integer
+                                inputs exact, empty groups give zeros
   gemm_nt_acc (+ _sampled)      pinned: integer inputs plus an integer C
                                 (exact), C alone (A = 0), the closed form
                                 C + float64 matmul, numpy's double->float32
@@ -74,6 +77,8 @@ def _load():
         lib.dgo_gemm_nt_acc.argtypes = [P, P, P, P, P, I, I, I, P, P]
         lib.dgo_gemm_nt_acc_sampled.restype = I
         lib.dgo_gemm_nt_acc_sampled.argtypes = [P, P, P, P, P, I, I, I, P, P, I64, P, P]
+        lib.dgo_k_grouped_tn.restype = I
+        lib.dgo_k_grouped_tn.argtypes = [P, P, P, P, P, I, I, I, I, P, P]
         lib.dgo_gemm_nt_sampled.restype = I
         lib.dgo_gemm_nt_sampled.argtypes = [P, P, P, P, I, I, I, P, P, I64, P, P]
         lib.dgo_grouped_contiguous.restype = I
@@ -202,6 +207,24 @@ def gemm_nt_acc_sampled(A, sA, B, sB, C, rows, cols):
     if rc:
         raise ValueError("dgo_gemm_nt_acc_sampled: bad sizes or indices")
     return o64, o32
+
+
+def k_grouped_tn(A, sA, B, sB, k_offsets, want_f64: bool = True):
+    """K-grouped TN GEMM: A [K][M], B [K][N] (MN-major), sA [K/128][M],
+    sB [K/128][N], k_offsets [G+1].  Returns (D64 or None, D32), [G][M][N]."""
+    A, B, sA, sB = _u8(A), _u8(B), _f32(sA), _f32(sB)
+    off = np.ascontiguousarray(k_offsets, dtype=np.int32)
+    K, M = A.shape
+    N = B.shape[1]
+    G = off.size - 1
+    assert B.shape[0] == K and sA.shape == (K // BLOCK, M) and sB.shape == (K // BLOCK, N)
+    d64 = np.empty((G, M, N), dtype=np.float64) if want_f64 else None
+    d32 = np.empty((G, M, N), dtype=np.float32)
+    rc = _load().dgo_k_grouped_tn(_ptr(A), _ptr(sA), _ptr(B), _ptr(sB), _ptr(off), G, M, N, K,
+                                  _ptr(d64), _ptr(d32))
+    if rc:
+        raise ValueError("dgo_k_grouped_tn: bad sizes or offsets")
+    return d64, d32
 
 
 def fp32_promotion_sampled(A, sA, B, sB, rows, cols):

@@ -238,6 +238,51 @@ int dgo_gemm_nt_acc_sampled(const uint8_t *A, const float *sA, const uint8_t *B,
     return 0;
 }
 
+/* K-grouped TN GEMM (the weight gradient of MoE experts): the hada.io
+ * page, section "Dense va Grouped GEMM", names a grouping along the K axis
+ * for MoE weight backward, with M and N fixed (k_grouped_fp8_gemm_tn_
+ * contiguous).  Group g owns K rows [off[g], off[g+1]) (multiples of 128) of
+ * A [K][M] and B [K][N], both stored MN-major (the TN layout), and
+ *
+ *   D_g[m,n] = sum_{kb in g} sA[kb,m] * sB[kb,n] * sum_{k in kb} dec(A[k,m]) * dec(B[k,n])
+ *
+ * with one fp32 scale per 128 rows of K and per column for both operands
+ * (sA [K/128][M], sB [K/128][N]: the scale granularity runs along the
+ * contraction, as the per-block promotion needs).  D is [G][M][N]; the sum
+ * is formed in double (block sums exact, as in dgo_gemm_nt) and rounded
+ * once to fp32.  An empty group gives zeros.  Returns -1 for bad offsets. */
+int dgo_k_grouped_tn(const uint8_t *A, const float *sA, const uint8_t *B,
+                     const float *sB, const int32_t *off, int G, int M, int N,
+                     int K, double *D64, float *D32)
+{
+    if (G <= 0 || M <= 0 || N <= 0 || K < 0 || K % DGO_BLOCK || off[0] != 0 || off[G] != K)
+        return -1;
+    for (int g = 0; g < G; ++g)
+        if (off[g + 1] < off[g] || off[g] % DGO_BLOCK)
+            return -1;
+    dgo_init_lut();
+#pragma omp parallel for schedule(dynamic, 1) collapse(2)
+    for (int g = 0; g < G; ++g) {
+        for (int m = 0; m < M; ++m) {
+            for (int n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int kb = off[g] / DGO_BLOCK; kb < off[g + 1] / DGO_BLOCK; ++kb) {
+                    double partial = 0.0;
+                    for (int k = kb * DGO_BLOCK; k < (kb + 1) * DGO_BLOCK; ++k)
+                        partial += g_lut[A[(int64_t)k * M + m]] * g_lut[B[(int64_t)k * N + n]];
+                    acc += (double)sA[(int64_t)kb * M + m] * (double)sB[(int64_t)kb * N + n] * partial;
+                }
+                const int64_t o = ((int64_t)g * M + m) * N + n;
+                if (D64)
+                    D64[o] = acc;
+                if (D32)
+                    D32[o] = (float)acc;
+            }
+        }
+    }
+    return 0;
+}
+
 /* Dense NT at selected (row, col) pairs only, for problems too large to
  * compute whole.  Same layouts as dgo_gemm_nt. */
 int dgo_gemm_nt_sampled(const uint8_t *A, const float *sA, const uint8_t *B,

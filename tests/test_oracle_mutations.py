@@ -38,6 +38,9 @@ MUTATIONS = {
     "bf16 truncation instead of round-to-nearest-even": (
         "double nq = nearbyint(r);",
         "double nq = floor(r);"),
+    "K-grouped: B scale of the wrong column block": (
+        "(double)sB[(int64_t)kb * N + n] * partial;",
+        "(double)sB[(int64_t)kb * N + n / 2] * partial;"),
     "accumulator C dropped from D = C + A.B^T": (
         "            double v = (double)C[(int64_t)m * N + n] +\n                       dgo_element(",
         "            double v = 0.0 * (double)C[(int64_t)m * N + n] +\n                       dgo_element("),
@@ -60,6 +63,8 @@ def _build_variant(tmp_path, old, new):
     lib.dgo_bf16_round.argtypes = [P, P, I64]
     lib.dgo_gemm_nt_acc.argtypes = [P, P, P, P, P, I, I, I, P, P]
     lib.dgo_gemm_nt_acc.restype = I
+    lib.dgo_k_grouped_tn.argtypes = [P, P, P, P, P, I, I, I, I, P, P]
+    lib.dgo_k_grouped_tn.restype = I
     return lib
 
 
@@ -108,7 +113,25 @@ def _pins_pass(lib) -> bool:
     e32 = np.empty((8, 128), np.float32)
     lib.dgo_gemm_nt_acc(_ptr(a8), _ptr(ones_a), _ptr(b8), _ptr(ones_b), _ptr(ci), 8, 128, 256,
                         _ptr(e64), _ptr(e32))
-    return bool(np.array_equal(e64, (ci + ai @ bi.T).astype(np.float64)))
+    if not np.array_equal(e64, (ci + ai @ bi.T).astype(np.float64)):
+        return False
+    # K-grouped: per-group float64 matmul of the dequantised slices
+    pk = gi.k_grouped_problem([128, 256], 24, 48, seed_a=28, seed_b=29)
+    off = pk["k_offsets"]
+    k64 = np.empty((2, 24, 48), np.float64)
+    k32 = np.empty((2, 24, 48), np.float32)
+    lib.dgo_k_grouped_tn(_ptr(np.ascontiguousarray(pk["A"])), _ptr(np.ascontiguousarray(pk["sA"])),
+                         _ptr(np.ascontiguousarray(pk["B"])), _ptr(np.ascontiguousarray(pk["sB"])),
+                         _ptr(off), 2, 24, 48, 384, _ptr(k64), _ptr(k32))
+    vals = lambda c: torch.from_numpy(np.ascontiguousarray(c)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ka = vals(pk["A"]) * np.repeat(pk["sA"].astype(np.float64), 128, axis=0)
+    kb = vals(pk["B"]) * np.repeat(pk["sB"].astype(np.float64), 128, axis=0)
+    for g in range(2):
+        ref = ka[off[g]:off[g + 1]].T @ kb[off[g]:off[g + 1]]
+        bound = np.abs(ka[off[g]:off[g + 1]]).T @ np.abs(kb[off[g]:off[g + 1]])
+        if not np.all(np.abs(k64[g] - ref) <= 1e-12 * bound + 1e-300):
+            return False
+    return True
 
 
 def test_unmutated_copy_passes(tmp_path):

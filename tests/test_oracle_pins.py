@@ -235,6 +235,45 @@ def test_acc_equals_c_plus_dequantised_matmul(oracle_mod):
     assert np.array_equal(s64, d64[r, q]) and np.array_equal(s32, d32[r, q])
 
 
+# ------------------------------------------------ K-grouped TN (wgrad)
+
+def test_k_grouped_equals_per_group_dequantised_matmul(oracle_mod):
+    # uneven groups, an empty group, M and N not multiples of 128
+    p = gi.k_grouped_problem([256, 0, 128, 384], 72, 144, seed_a=25, seed_b=26)
+    d64, d32 = oracle_mod.k_grouped_tn(p["A"], p["sA"], p["B"], p["sB"], p["k_offsets"])
+    vals = lambda c: torch.from_numpy(np.ascontiguousarray(c)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    a = vals(p["A"]) * np.repeat(p["sA"].astype(np.float64), BLOCK, axis=0)  # [K][M]
+    b = vals(p["B"]) * np.repeat(p["sB"].astype(np.float64), BLOCK, axis=0)  # [K][N]
+    off = p["k_offsets"]
+    for g in range(p["G"]):
+        ag, bg = a[off[g]:off[g + 1]], b[off[g]:off[g + 1]]
+        ref = ag.T @ bg
+        bound = np.abs(ag).T @ np.abs(bg)
+        assert np.all(np.abs(d64[g] - ref) <= 1e-12 * bound + 1e-300), g
+    assert np.all(d64[1] == 0.0)  # the empty group
+    assert np.array_equal(d32.view(np.uint32), d64.astype(np.float32).view(np.uint32))
+
+
+def test_k_grouped_integer_inputs_exact(oracle_mod):
+    rng = np.random.default_rng(27)
+    ks, M, N = [128, 256], 40, 64
+    K = sum(ks)
+    ai, bi = rng.integers(-4, 5, (K, M)), rng.integers(-4, 5, (K, N))
+    to8 = lambda x: torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    off = np.array([0, 128, 384], np.int32)
+    _, d32 = oracle_mod.k_grouped_tn(to8(ai), np.ones((K // BLOCK, M), np.float32), to8(bi),
+                                     np.ones((K // BLOCK, N), np.float32), off)
+    assert np.array_equal(d32[0], (ai[:128].T @ bi[:128]).astype(np.float32))
+    assert np.array_equal(d32[1], (ai[128:].T @ bi[128:]).astype(np.float32))
+
+
+def test_k_grouped_rejects_bad_offsets(oracle_mod):
+    p = gi.k_grouped_problem([128, 128], 16, 16)
+    for bad in ([0, 100, 256], [0, 256, 128], [0, 128, 384]):
+        with pytest.raises(ValueError):
+            oracle_mod.k_grouped_tn(p["A"], p["sA"], p["B"], p["sB"], np.array(bad, np.int32))
+
+
 # ----------------------------------------------------------------- grouped
 
 SENTINEL = 0x7FC1  # a NaN pattern nobody computes
