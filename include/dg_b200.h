@@ -117,6 +117,34 @@ dg_status_t dg_fp8_gemm_tt(const void *A, const float *sA, const void *B,
                            cudaStream_t stream);
 
 /*
+ * K-grouped TN GEMM for MoE weight gradients (hada.io page, section "Dense
+ * va Grouped GEMM": a grouping along the K axis, M and N fixed, named
+ * k_grouped_fp8_gemm_tn_contiguous).  Group g owns K rows
+ * [k_offsets[g], k_offsets[g+1]) of the shared K axis and
+ *   D[g] = A[rows of g]^T @ B[rows of g],  D[g][m][n] fp32.
+ *   A         : [K][M]  e4m3, M-major (M % 16 == 0)
+ *   sA        : [K/128][M_pad] fp32, one scale per 128 rows of K and per m,
+ *               M_pad = dg_get_tma_aligned_size(M, 4)
+ *   B         : [K][N]  e4m3, N-major
+ *   sB        : [K/128][N] fp32, one scale per 128 rows of K and per n
+ *               (16-byte aligned)
+ *   D         : [G][M][N] fp32, written whole (an empty group gives zeros)
+ *   k_offsets : [G+1] int32 DEVICE array, k_offsets[0] = 0, non-decreasing
+ *               multiples of 128, k_offsets[G] = K; read only on the device
+ *               (a malformed group is computed as empty and flagged with
+ *               DG_ERR_BAD_GROUP_DATA in the status word)
+ * The pages give neither the scale granularity nor the output type: scales
+ * per 128 K rows and per column of both operands (the granularity along the
+ * contraction that per-block promotion needs) and an fp32 output are the
+ * readings taken.  K == 0 zero-fills D.  Runs on one-CTA tiles of 128 or 256
+ * columns.
+ */
+dg_status_t dg_fp8_k_grouped_gemm_tn_contiguous(const void *A, const float *sA, const void *B,
+                                                const float *sB, float *D,
+                                                const int32_t *k_offsets, int M, int N, int K,
+                                                int num_groups, cudaStream_t stream);
+
+/*
  * Dense NT GEMM with an accumulator: D = C + A @ B^T, the "D = C + A @ B"
  * form of the pages (hada.io page, section "Giao dien GEMM va rang buoc
  * layout": fp8_gemm_nt computes D = C + A @ B.T).  The pages give C no

@@ -40,6 +40,7 @@ _I = ctypes.c_int
 _SIGNATURES = {
     "dg_fp8_gemm_nt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_nt_acc": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "dg_fp8_k_grouped_gemm_tn_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_fp8_gemm_nn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_tn": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_gemm_tt": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
@@ -270,6 +271,32 @@ def dg_fp8_gemm_tn(A, sA, B, sB, D, stream=None) -> None:
 def dg_fp8_gemm_tt(A, sA, B, sB, D, stream=None) -> None:
     """D = A^T @ B^T with A stored [K, M] (M-major) and B stored [N, K]."""
     _dense_layout("dg_fp8_gemm_tt", True, False, A, sA, B, sB, D, stream)
+
+
+def dg_fp8_k_grouped_gemm_tn_contiguous(A, sA, B, sB, D, k_offsets, stream=None) -> None:
+    """D[g] = A[K rows of g]^T @ B[K rows of g]: A [K, M], B [K, N] (MN-major),
+    sA [K/128, M_pad], sB [K/128, N], D [G, M, N] float32, k_offsets [G+1]
+    int32 on the device."""
+    pa = _dev(A, "A", _FP8, 2)
+    K, M = A.shape
+    pb = _dev(B, "B", _FP8, 2)
+    if B.shape[0] != K:
+        raise ValueError("B must be [K, N]")
+    N = B.shape[1]
+    psa = _dev(sA, "sA", _F32, 2)
+    if tuple(sA.shape) != (K // 128, get_tma_aligned_size(M, 4)):
+        raise ValueError(f"sA must be [K/128, M_pad] = {(K // 128, get_tma_aligned_size(M, 4))}")
+    psb = _dev(sB, "sB", _F32, 2)
+    if tuple(sB.shape) != (K // 128, N):
+        raise ValueError("sB must be [K/128, N]")
+    po = _dev(k_offsets, "k_offsets", (torch.int32,), 1)
+    G = k_offsets.shape[0] - 1
+    pd = _dev(D, "D", _F32, 3)
+    if tuple(D.shape) != (G, M, N):
+        raise ValueError("D must be [G, M, N]")
+    st = load_library().dg_fp8_k_grouped_gemm_tn_contiguous(pa, psa, pb, psb, pd, po, M, N, K, G,
+                                                            _stream_handle(stream, A.device))
+    _check("dg_fp8_k_grouped_gemm_tn_contiguous", st)
 
 
 def dg_fp8_gemm_nt_acc(A, sA, B, sB, C, D, stream=None) -> None:

@@ -321,7 +321,7 @@ template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false,
 dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
                           const GemmParams &p, int grid, cudaStream_t stream)
 {
-    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT>;
+    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == dg::kKGrouped>;
     CUtensorMap ta, tb;
     const bool ok_a = A_MN ? make_tmap_mn(&ta, A, a_rows, static_cast<uint64_t>(p.K), KS * dg::kBK)
                            : make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS);
@@ -540,7 +540,7 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
     }
     p.ksplit = plan.ksplit;
     p.kb_per_split = (p.num_kb + plan.ksplit - 1) / plan.ksplit;
-    const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
+    const int64_t tiles = static_cast<int64_t>(LAYOUT == dg::kKGrouped ? p.G : 1) * p.num_mb * p.num_nb;
     if (plan.ksplit > 1) {
         const size_t bytes = static_cast<size_t>(tiles) * plan.ksplit * c.bn * dg::kBM * sizeof(float);
         void *ws = nullptr;
@@ -667,6 +667,61 @@ dg_status_t dg_fp8_gemm_tt(const void *A, const float *sA, const void *B, const 
                            void *D, int M, int N, int K, cudaStream_t stream)
 {
     return dense_gemm(A, sA, B, sB, D, M, N, K, true, false, stream);
+}
+
+dg_status_t dg_fp8_k_grouped_gemm_tn_contiguous(const void *A, const float *sA, const void *B,
+                                                const float *sB, float *D, const int32_t *k_offsets,
+                                                int M, int N, int K, int num_groups, cudaStream_t stream)
+{
+    if (!A || !sA || !B || !sB || !D || !k_offsets || M < 0 || N <= 0 || K < 0 || num_groups <= 0)
+        return DG_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N % 16 != 0 || M % 16 != 0)
+        return DG_ERR_UNSUPPORTED;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sA, 16) ||
+        !aligned(sB, 16) || !aligned(k_offsets, 4))
+        return DG_ERR_ALIGNMENT;
+    if (static_cast<int64_t>(num_groups) * M * N > 0x7FFFFFFFll * 4)
+        return DG_ERR_UNSUPPORTED;
+    if (M == 0)
+        return DG_OK;
+    if (K == 0) {
+        // every group is empty: each D_g is zero
+        if (cudaMemsetAsync(D, 0, static_cast<size_t>(num_groups) * M * N * sizeof(float), stream) !=
+            cudaSuccess) {
+            (void)cudaGetLastError();
+            return DG_ERR_CUDA;
+        }
+        return DG_OK;
+    }
+    const int dev = current_device();
+    const int sms = effective_sms(dev);
+    if (sms <= 0)
+        return DG_ERR_CUDA;
+    GemmParams p{};
+    p.sA = sA;
+    p.sB = sB;
+    p.D = reinterpret_cast<__nv_bfloat16 *>(D);  // shapes the unused store tensor maps only
+    p.D32 = D;
+    p.k_offsets = k_offsets;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = num_groups;
+    p.sa_ld = dg_get_tma_aligned_size(M, 4);
+    p.num_kb = K / 128;
+    p.nbn = (N + 127) / 128;
+    p.num_mb = (M + 127) / 128;
+    p.raster = 1;
+    p.timeout_ns = g_timeout_ns.load();
+    p.stall_injection = g_stall_injection.load();
+    const int avg_kb = p.num_kb / num_groups > 0 ? p.num_kb / num_groups : 1;
+    const Plan plan = choose_plan(static_cast<int64_t>(num_groups) * p.num_mb, 0, N, avg_kb, sms, false,
+                                  kNoPair | kWholeBoxes);
+    if (print_configs())
+        std::fprintf(stderr, "[dg] k-grouped tn G=%d M=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
+                     num_groups, M, N, K, plan.c.bn, plan.c.stages, plan.c.ks, sms);
+    return dispatch<dg::kKGrouped, true, true>(plan, A, static_cast<uint64_t>(M), B,
+                                                static_cast<uint64_t>(N), p, sms, stream);
 }
 
 dg_status_t dg_fp8_gemm_nt_acc(const void *A, const float *sA, const void *B, const float *sB,

@@ -57,7 +57,9 @@
 
 namespace dg {
 
-enum Layout : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+// kKGrouped: the K-grouped TN GEMM (MoE weight gradient): groups own
+// 128-row segments of the shared K axis, D is fp32 [G][M][N].
+enum Layout : int { kDense = 0, kContiguous = 1, kMasked = 2, kKGrouped = 3 };
 
 // Device status word: code (bits 0-7), role (8-11), stage (12-19), CTA (20-31).
 constexpr uint32_t kCodeTimeout = 5;
@@ -96,7 +98,19 @@ struct GemmParams {
     // fp32 D32[M][N] = C[M][N] + acc (C may be D32 itself) instead of bf16 D.
     const float *C;
     float *D32;
+    const int32_t *k_offsets;  // K-grouped only: [G+1] K-row offsets of the groups
 };
+
+// Row segment of an fp32 output: drow[c] = acc[c] for the 4-float groups of
+// this thread's row that lie inside N.
+template <int COLS>
+__device__ __forceinline__ void store_row_f32(float *drow, const float *acc, int col0, int N)
+{
+#pragma unroll
+    for (int c = 0; c < COLS; c += 4)
+        if (col0 + c < N)
+            *reinterpret_cast<float4 *>(drow + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+}
 
 // Row segment of the accumulate form: drow[c] = crow[c] + acc[c] for the
 // 4-float groups of this thread's row that lie inside N (read before write,
@@ -142,16 +156,41 @@ struct TileScheduler {
     // This CTA's K blocks: [begin, end).
     __device__ int kb_begin() const
     {
+        if constexpr (LAYOUT == kKGrouped)
+            return cur_kb0;
         return p.ksplit > 1 ? static_cast<int>(blockIdx.x % p.ksplit) * p.kb_per_split : 0;
     }
     __device__ int kb_end() const
     {
+        if constexpr (LAYOUT == kKGrouped)
+            return cur_kb1;
         return p.ksplit > 1 ? min(p.num_kb, kb_begin() + p.kb_per_split) : p.num_kb;
     }
+    int cur_kb0 = 0, cur_kb1 = 0;  // K-grouped: the current tile's K blocks
 
     __device__ bool next(TileCoord &tc, bool report)
     {
-        if constexpr (LAYOUT == kMasked) {
+        if constexpr (LAYOUT == kKGrouped) {
+            // tiles group by group, each group's m-blocks fastest
+            const int per_group = p.num_mb * p.num_nb;
+            const int t = next_t;
+            if (t >= p.G * per_group)
+                return false;
+            next_t += stride;
+            tc.g = t / per_group;
+            const int within = t - tc.g * per_group;
+            tc.nb = within / p.num_mb;
+            tc.mb = within - tc.nb * p.num_mb;
+            int k0 = __ldg(p.k_offsets + tc.g), k1 = __ldg(p.k_offsets + tc.g + 1);
+            if (k0 < 0 || k1 < k0 || k1 > p.K || (k0 % kBK) || (k1 % kBK)) {
+                if (report)
+                    record_status(kCodeBadGroup, kRoleSched, tc.g);
+                k0 = k1 = 0;  // a malformed group is computed as empty
+            }
+            cur_kb0 = k0 / kBK;
+            cur_kb1 = k1 / kBK;
+            return true;
+        } else if constexpr (LAYOUT == kMasked) {
             const int t = next_t;
             while (true) {
                 if (cur_g >= p.G)
@@ -249,8 +288,11 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
 // BN: tile width; STAGES: shared-memory ring depth; KS: 128-wide K blocks per
 // stage (one 3-D TMA box per operand carries all KS blocks -- the TMA engine
 // costs a roughly fixed time per instruction, so bigger boxes move more).
-template <int BN_, int STAGES_, int KS_, bool SPLIT_ = false>
+template <int BN_, int STAGES_, int KS_, bool SPLIT_ = false, bool COLSCALE_ = false>
 struct KernelConfig {
+    // COLSCALE: one B scale per column and K block (the K-grouped layout)
+    // instead of one per 128x128 block.
+    static constexpr bool COLSCALE = COLSCALE_;
     static constexpr int BN = BN_;
     static constexpr int STAGES = STAGES_;
     static constexpr int KS = KS_;
@@ -274,7 +316,8 @@ struct KernelConfig {
     static constexpr int B_BYTES = BN * kBK;   // one K block of B
     static constexpr int STAGE_BYTES = KS * (A_BYTES + B_BYTES);
     static constexpr int SA_BYTES = KS * kBM * 4;  // LHS scales of a stage
-    static constexpr int SB_BYTES = KS * 16;       // up to 3 weight-block scales per K block
+    static constexpr int SB_FLOATS = COLSCALE ? BN : 4;  // B scales per K block
+    static constexpr int SB_BYTES = KS * SB_FLOATS * 4;  // (at most 3 weight-block scales, or BN columns)
     // TMEM: NBUF partial buffers of ACC_STRIDE columns (<= 512 in total), so
     // the MMA can run NBUF-1 K blocks ahead of the promotion.
     static constexpr int ACC_STRIDE = (BN + 31) / 32 * 32;
@@ -345,15 +388,17 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float *v)
 // bytes by 128*KS K rows (B: one box per 128 columns, BN % 128 == 0) and
 // described to the MMA as an MN-major 128-byte-swizzled operand.
 template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false>
-__global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 1)
+__global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped>::THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d64,
                     const __grid_constant__ CUtensorMap tmap_drem, const GemmParams p)
 {
-    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT>;
+    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped>;
     static_assert(!SPLIT || LAYOUT == kDense, "K split is implemented for the dense layout");
-    static_assert((!A_MN && !B_MN) || LAYOUT == kDense, "MN-major operands are implemented for the dense layout");
+    static_assert((!A_MN && !B_MN) || LAYOUT == kDense || LAYOUT == kKGrouped,
+                  "MN-major operands are implemented for the dense and K-grouped layouts");
+    static_assert(LAYOUT != kKGrouped || (A_MN && B_MN), "the K-grouped GEMM is the TN layout");
     static_assert(!B_MN || BN % 128 == 0, "an MN-major B tile is whole 128-column boxes");
     constexpr int BN_WG = Cfg::BN_WG;
     constexpr int RMAX = Cfg::RMAX;
@@ -365,8 +410,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
     uint8_t *a_tiles = smem;                                   // [STAGES*KS][128][128 B]
     uint8_t *b_tiles = smem + STAGES * KS * Cfg::A_BYTES;      // [STAGES*KS][BN][128 B]
     float *sa_tiles = reinterpret_cast<float *>(smem + STAGES * Cfg::STAGE_BYTES);  // [STAGES*KS][128]
-    float *sb_tiles = sa_tiles + STAGES * KS * kBM;            // [STAGES*KS][4]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sb_tiles + STAGES * KS * 4);
+    float *sb_tiles = sa_tiles + STAGES * KS * kBM;            // [STAGES*KS][SB_FLOATS]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sb_tiles + STAGES * KS * Cfg::SB_FLOATS);
     uint64_t *full_bar = bars;                 // stage landed (TMA bytes + scale copies)
     uint64_t *empty_bar = bars + STAGES;       // MMAs of the stage done (operand tiles free)
     uint64_t *sread_bar = bars + 2 * STAGES;   // promotion warps have read the stage's scales
@@ -428,7 +473,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
         bool ok = !(p.stall_injection && blockIdx.x == 0);
         while (ok && sched.next(tc, lane == 0)) {
             const int a_row = (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * kBM;
-            const int b_row = tc.g * p.N + tc.nb * BN;
+            // (the K-grouped layout shares one B across its groups)
+            const int b_row = (LAYOUT == kKGrouped ? 0 : tc.g * p.N) + tc.nb * BN;
             const int m0 = tc.mb * kBM;
             const float *sa_base = p.sA +
                                    (LAYOUT == kMasked ? static_cast<size_t>(tc.g) * p.num_kb * p.sa_ld : 0) +
@@ -477,9 +523,23 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                                 sa_ok ? static_cast<const void *>(sa_base + static_cast<size_t>(kb) * p.sa_ld)
                                       : static_cast<const void *>(p.sA),
                                 sa_ok ? 16u : 0u);
-                    if (lane < 3)
-                        cp_async_4(smem_addr(sb_tiles + (stage * KS + q) * 4) + 4 * lane,
-                                   sb_src + (in_k ? kb : kb_end - 1));
+                    if constexpr (Cfg::COLSCALE) {
+                        // the tile's BN column scales of this K block, in
+                        // 16-byte pieces (zeros past N)
+#pragma unroll
+                        for (int c4 = lane; c4 < BN / 4; c4 += 32) {
+                            const int col = tc.nb * BN + 4 * c4;
+                            const bool ok_c = in_k && col < p.N;
+                            cp_async_16(smem_addr(sb_tiles + (stage * KS + q) * BN) + 16 * c4,
+                                        ok_c ? static_cast<const void *>(p.sB + static_cast<size_t>(kb) * p.N + col)
+                                             : static_cast<const void *>(p.sB),
+                                        ok_c ? 16u : 0u);
+                        }
+                    } else {
+                        if (lane < 3)
+                            cp_async_4(smem_addr(sb_tiles + (stage * KS + q) * 4) + 4 * lane,
+                                       sb_src + (in_k ? kb : kb_end - 1));
+                    }
                 }
                 cp_async_mbar_arrive_noinc(fb);
                 __syncwarp();
@@ -594,7 +654,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
         while (ok && sched.next(tc, false)) {
             const int m_local = tc.mb * kBM + row;  // row index inside the group
             bool row_ok;
-            if constexpr (LAYOUT == kDense) {
+            if constexpr (LAYOUT == kDense || LAYOUT == kKGrouped) {
                 row_ok = m_local < p.M;
             } else if constexpr (LAYOUT == kContiguous) {
                 row_ok = false;
@@ -628,15 +688,25 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                     break;
                 }
                 float s_lo[KS], s_hi[KS];
+                // column scales (K-grouped): read per element below, so the
+                // scale slots are handed back after the stage's K blocks
+                const float *sb_cols = sb_tiles + stage * KS * Cfg::SB_FLOATS + wg * BN_WG;
+                const uint32_t stage_of_scales = stage;
 #pragma unroll
                 for (int q = 0; q < KS; ++q) {
                     const float sa = sa_tiles[(stage * KS + q) * kBM + row];
-                    s_lo[q] = sa * sb_tiles[(stage * KS + q) * 4 + j_lo];
-                    s_hi[q] = sa * sb_tiles[(stage * KS + q) * 4 + j_hi];
+                    if constexpr (Cfg::COLSCALE) {
+                        s_lo[q] = s_hi[q] = sa;
+                    } else {
+                        s_lo[q] = sa * sb_tiles[(stage * KS + q) * 4 + j_lo];
+                        s_hi[q] = sa * sb_tiles[(stage * KS + q) * 4 + j_hi];
+                    }
                 }
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(smem_addr(sread_bar + stage));
+                if constexpr (!Cfg::COLSCALE) {
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(smem_addr(sread_bar + stage));
+                }
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
@@ -673,14 +743,31 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
 #pragma unroll
                         for (int g8 = 0; g8 < RMAX; g8 += 8) {
                             if (whole || g8 < TAIL) {
-                                const float sc = (c0 + g8 >= boundary) ? s_hi[q] : s_lo[q];
+                                if constexpr (Cfg::COLSCALE) {
+                                    // sA[kb,m] * sB[kb,n] per column (a
+                                    // broadcast shared-memory read)
+                                    const float *sbq = sb_cols + q * Cfg::SB_FLOATS + c0 + g8;
 #pragma unroll
-                                for (int i = 0; i < 8; ++i)
-                                    acc[c0 + g8 + i] = fmaf(__uint_as_float(r[g8 + i]), sc, acc[c0 + g8 + i]);
+                                    for (int i = 0; i < 8; ++i)
+                                        acc[c0 + g8 + i] = fmaf(__uint_as_float(r[g8 + i]), s_lo[q] * sbq[i],
+                                                                acc[c0 + g8 + i]);
+                                } else {
+                                    const float sc = (c0 + g8 >= boundary) ? s_hi[q] : s_lo[q];
+#pragma unroll
+                                    for (int i = 0; i < 8; ++i)
+                                        acc[c0 + g8 + i] = fmaf(__uint_as_float(r[g8 + i]), sc, acc[c0 + g8 + i]);
+                                }
                             }
                         }
                     }
                     ++acc_i;
+                }
+                if constexpr (Cfg::COLSCALE) {
+                    if (ok) {
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(smem_addr(sread_bar + stage_of_scales));
+                    }
                 }
                 if (!ok)
                     break;
@@ -722,6 +809,13 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT>::THREADS, 
                                                  p.N);
                     continue;
                 }
+            }
+            if constexpr (LAYOUT == kKGrouped) {
+                // fp32 D_g, row by row
+                if (row_ok)
+                    store_row_f32<BN_WG>(p.D32 + (static_cast<size_t>(tc.g) * p.M + m_local) * p.N + col0, acc,
+                                         col0, p.N);
+                continue;
             }
             const bool tile_rows_ok = named_barrier_and(
                 1 + wg, 128, LAYOUT == kDense ? (tc.mb * kBM < p.M) : row_ok);

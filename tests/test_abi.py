@@ -87,6 +87,14 @@ def test_null_and_alignment(lib):
     assert lib.dg_fp8_gemm_tt(FAKE, FAKE, FAKE, FAKE, FAKE, 200, 256, 512, None) == 2
     assert lib.dg_fp8_gemm_nn(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 250, 512, None) == 2
     assert lib.dg_fp8_gemm_nn(None, FAKE, FAKE, FAKE, FAKE, 128, 256, 512, None) == 1
+    # K-grouped TN: sizes, alignment, group count
+    kg = lib.dg_fp8_k_grouped_gemm_tn_contiguous
+    assert kg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 512, 0, None) == 1
+    assert kg(FAKE, FAKE, FAKE, FAKE, FAKE, None, 128, 256, 512, 2, None) == 1
+    assert kg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 120, 256, 512, 2, None) == 2
+    assert kg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 500, 2, None) == 2
+    assert kg(FAKE, FAKE, FAKE, odd, FAKE, FAKE, 128, 256, 512, 2, None) == 3
+    assert kg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 512, 2, None) == 0
     # accumulate form: C is required and 16-byte aligned; same shape rules
     assert lib.dg_fp8_gemm_nt_acc(FAKE, FAKE, FAKE, FAKE, None, FAKE, 128, 256, 512, None) == 1
     assert lib.dg_fp8_gemm_nt_acc(FAKE, FAKE, FAKE, FAKE, odd, FAKE, 128, 256, 512, None) == 3
