@@ -13,7 +13,11 @@ shapes; no dataset or weights are used, these synthetic tensors stand in):
     scale = max(amax, 1e-4) / 448 in float32 (a partial last block of B's
     rows counts only its real rows);
   * codes = e4m3fn(clamp(x / scale, -448, 448)), cast by torch on the CPU
-    (round to nearest even; the clamp makes the cast saturating).
+    (round to nearest even; the clamp makes the cast saturating);
+  * UE8M0 inputs (``ue8m0=True``, the SM100 block-scaled mode: hada.io
+    DeepGEMM summary, "Giao dien GEMM va rang buoc layout") take instead the
+    smallest power of two scale >= max(amax, 1e-4) / 448, decided in float64,
+    and quantise the data with it.
 Fine-grained 1x128 / 128x128 scaling: "deepseek开源周第三天：DeepGEMM深度分析"
 (pxiaoer.blog), FP8-training list.
 
@@ -46,18 +50,29 @@ def _cast_e4m3(y: np.ndarray) -> np.ndarray:
         torch.float8_e4m3fn).view(torch.uint8).numpy()
 
 
-def quantize_1x128(x: np.ndarray):
+def _block_scale(amax: np.ndarray, ue8m0: bool) -> np.ndarray:
+    """Scale of each block from its amax: amax/448 in float32, or with
+    ue8m0 the smallest power of two >= amax/448 (in float64: x = f * 2**e
+    with 0.5 <= f < 1 is itself a power of two iff f == 0.5)."""
+    if not ue8m0:
+        return (np.maximum(amax, np.float32(AMAX_FLOOR)) / np.float32(E4M3_MAX)).astype(np.float32)
+    ratio = np.maximum(amax.astype(np.float64), AMAX_FLOOR) / E4M3_MAX
+    frac, expo = np.frexp(ratio)
+    return np.where(frac == 0.5, ratio, np.ldexp(1.0, expo)).astype(np.float32)
+
+
+def quantize_1x128(x: np.ndarray, ue8m0: bool = False):
     """x: [..., K] float32 -> (codes uint8 [..., K], scales float32 [..., K/128])."""
     *lead, K = x.shape
     assert K % BLOCK == 0
     xb = x.reshape(*lead, K // BLOCK, BLOCK)
     amax = np.abs(xb).max(axis=-1)
-    scale = (np.maximum(amax, np.float32(AMAX_FLOOR)) / np.float32(E4M3_MAX)).astype(np.float32)
+    scale = _block_scale(amax, ue8m0)
     y = xb / scale[..., None]
     return _cast_e4m3(y).reshape(x.shape), scale
 
 
-def quantize_128x128(x: np.ndarray):
+def quantize_128x128(x: np.ndarray, ue8m0: bool = False):
     """x: [N, K] float32 -> (codes uint8 [N, K], scales float32 [ceil(N/128), K/128])."""
     N, K = x.shape
     assert K % BLOCK == 0
@@ -69,7 +84,7 @@ def quantize_128x128(x: np.ndarray):
         r = rows.shape[0]
         xb = rows.reshape(r, K // BLOCK, BLOCK)
         amax = np.abs(xb).max(axis=(0, 2))
-        s = (np.maximum(amax, np.float32(AMAX_FLOOR)) / np.float32(E4M3_MAX)).astype(np.float32)
+        s = _block_scale(amax, ue8m0)
         scales[nb] = s
         codes[nb * BLOCK:(nb + 1) * BLOCK] = _cast_e4m3(xb / s[None, :, None]).reshape(r, K)
     return codes, scales
@@ -108,19 +123,20 @@ def sa_to_kernel_layout(sa_logical: np.ndarray) -> np.ndarray:
 
 # ----------------------------------------------------------- problem recipes
 
-def dense_problem(M: int, N: int, K: int, seed_a: int = SEED_A, seed_b: int = SEED_B):
-    a, sa = quantize_1x128(standard_normal(seed_a, (M, K)))
-    b, sb = quantize_128x128(standard_normal(seed_b, (N, K)))
+def dense_problem(M: int, N: int, K: int, seed_a: int = SEED_A, seed_b: int = SEED_B,
+                  ue8m0: bool = False):
+    a, sa = quantize_1x128(standard_normal(seed_a, (M, K)), ue8m0)
+    b, sb = quantize_128x128(standard_normal(seed_b, (N, K)), ue8m0)
     return dict(kind="dense", A=a, sA=sa, B=b, sB=sb, M=M, N=N, K=K)
 
 
-def grouped_weights(G: int, N: int, K: int, seed_b: int = SEED_B):
+def grouped_weights(G: int, N: int, K: int, seed_b: int = SEED_B, ue8m0: bool = False):
     gen = np.random.Generator(np.random.PCG64(seed_b))
     nbn = (N + BLOCK - 1) // BLOCK
     B = np.empty((G, N, K), dtype=np.uint8)
     sB = np.empty((G, nbn, K // BLOCK), dtype=np.float32)
     for g in range(G):
-        B[g], sB[g] = quantize_128x128(gen.standard_normal((N, K), dtype=np.float32))
+        B[g], sB[g] = quantize_128x128(gen.standard_normal((N, K), dtype=np.float32), ue8m0)
     return B, sB
 
 
@@ -138,7 +154,7 @@ def k_grouped_problem(ks, M: int, N: int, seed_a: int = SEED_A, seed_b: int = SE
 
 
 def contiguous_problem(rows_per_group, N: int, K: int, seed_a: int = SEED_A,
-                       seed_b: int = SEED_B, pad_to: int = BLOCK):
+                       seed_b: int = SEED_B, pad_to: int = BLOCK, ue8m0: bool = False):
     """Contiguous grouped layout.  Group g's segment has rows_per_group[g]
     real rows, padded up to a multiple of ``pad_to`` with rows tagged -1."""
     G = len(rows_per_group)
@@ -148,8 +164,8 @@ def contiguous_problem(rows_per_group, N: int, K: int, seed_a: int = SEED_A,
         idx += [g] * r + [-1] * (padded - r)
     m_indices = np.asarray(idx, dtype=np.int32)
     M = m_indices.size
-    a, sa = quantize_1x128(standard_normal(seed_a, (M, K)))
-    B, sB = grouped_weights(G, N, K, seed_b)
+    a, sa = quantize_1x128(standard_normal(seed_a, (M, K)), ue8m0)
+    B, sB = grouped_weights(G, N, K, seed_b, ue8m0)
     return dict(kind="contiguous", A=a, sA=sa, B=B, sB=sB, m_indices=m_indices,
                 M=M, N=N, K=K, G=G)
 
@@ -160,12 +176,13 @@ def masked_counts(G: int, max_m: int, seed: int = SEED_MASK, low: int = 1):
 
 
 def masked_problem(G: int, max_m: int, N: int, K: int, masked_m=None,
-                   seed_a: int = SEED_A, seed_b: int = SEED_B, seed_mask: int = SEED_MASK):
+                   seed_a: int = SEED_A, seed_b: int = SEED_B, seed_mask: int = SEED_MASK,
+                   ue8m0: bool = False):
     if masked_m is None:
         masked_m = masked_counts(G, max_m, seed_mask)
     masked_m = np.asarray(masked_m, dtype=np.int32)
-    a, sa = quantize_1x128(standard_normal(seed_a, (G, max_m, K)))
-    B, sB = grouped_weights(G, N, K, seed_b)
+    a, sa = quantize_1x128(standard_normal(seed_a, (G, max_m, K)), ue8m0)
+    B, sB = grouped_weights(G, N, K, seed_b, ue8m0)
     return dict(kind="masked", A=a, sA=sa, B=B, sB=sB, masked_m=masked_m,
                 G=G, max_m=max_m, N=N, K=K)
 
@@ -180,10 +197,10 @@ WORKLOADS = {
 }
 
 
-def make_workload(name: str):
+def make_workload(name: str, ue8m0: bool = False):
     w = WORKLOADS[name]
     if w["kind"] == "dense":
-        return dense_problem(w["M"], w["N"], w["K"])
+        return dense_problem(w["M"], w["N"], w["K"], ue8m0=ue8m0)
     if w["kind"] == "contiguous":
-        return contiguous_problem([w["rows"]] * w["G"], w["N"], w["K"])
-    return masked_problem(w["G"], w["max_m"], w["N"], w["K"])
+        return contiguous_problem([w["rows"]] * w["G"], w["N"], w["K"], ue8m0=ue8m0)
+    return masked_problem(w["G"], w["max_m"], w["N"], w["K"], ue8m0=ue8m0)

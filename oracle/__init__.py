@@ -27,6 +27,14 @@ Parity status of each function (what pins it is listed in the tests):
                                 untouched padding / masked rows
   fp32_promotion_sampled        analysis aid (not a reference), pinned against
                                 a float32 re-computation on small cases
+  ue8m0_value / ue8m0_from_scale  pinned: every code vs Python's exact 2.0**k,
+                                round trip of all 255 finite codes, rejection
+                                of non-powers of two, zero, inf, NaN, range
+  ue8m0_ceil_pow2               pinned: a doubling/halving search (no frexp)
+                                on random and boundary values, exact powers
+  pack_ue8m0 / unpack_ue8m0     pinned: a hand-worked example (byte j = K
+                                block 4g+j, pad 127), round trip
+  gemm_nt_ue8m0 (+ grouped)     the GEMM above on the unpacked scales
 """
 from __future__ import annotations
 
@@ -77,6 +85,16 @@ def _load():
         lib.dgo_gemm_nt_acc.argtypes = [P, P, P, P, P, I, I, I, P, P]
         lib.dgo_gemm_nt_acc_sampled.restype = I
         lib.dgo_gemm_nt_acc_sampled.argtypes = [P, P, P, P, P, I, I, I, P, P, I64, P, P]
+        lib.dgo_ue8m0_value.restype = ctypes.c_double
+        lib.dgo_ue8m0_value.argtypes = [ctypes.c_uint8]
+        lib.dgo_ue8m0_from_scale.restype = I
+        lib.dgo_ue8m0_from_scale.argtypes = [ctypes.c_double]
+        lib.dgo_ue8m0_ceil_pow2.restype = ctypes.c_double
+        lib.dgo_ue8m0_ceil_pow2.argtypes = [ctypes.c_double]
+        lib.dgo_pack_ue8m0.restype = I
+        lib.dgo_pack_ue8m0.argtypes = [P, I, I, P]
+        lib.dgo_unpack_ue8m0.restype = I
+        lib.dgo_unpack_ue8m0.argtypes = [P, I, I, P]
         lib.dgo_k_grouped_tn.restype = I
         lib.dgo_k_grouped_tn.argtypes = [P, P, P, P, P, I, I, I, I, P, P]
         lib.dgo_gemm_nt_sampled.restype = I
@@ -280,3 +298,75 @@ def grouped_masked(A, sA, B, sB, masked_m, D16_init, want_f64=False):
     if rc:
         raise ValueError("dgo_grouped_masked: bad sizes")
     return d64, d16
+
+
+# ------------------------------------------------------------ UE8M0 scales
+
+def ue8m0_value(code: int) -> float:
+    """UE8M0 code -> 2**(code-127); 255 is NaN."""
+    return _load().dgo_ue8m0_value(int(code))
+
+
+def ue8m0_from_scale(s: float) -> int:
+    """Exact code of a power-of-two scale in [2**-127, 2**127], else -1."""
+    return _load().dgo_ue8m0_from_scale(float(s))
+
+
+def ue8m0_ceil_pow2(x: float) -> float:
+    """Smallest power of two >= x (finite x > 0): the UE8M0 scale of a block
+    is ue8m0_ceil_pow2(amax / 448)."""
+    return _load().dgo_ue8m0_ceil_pow2(float(x))
+
+
+def pack_ue8m0(s):
+    """s: [..., rows, nkb] fp32 powers of two -> [..., ceil(nkb/4), rows]
+    int32, byte j of word (g, r) = code of K block 4g+j (127 past nkb)."""
+    s = _f32(s)
+    *lead, rows, nkb = s.shape
+    ng = (nkb + 3) // 4
+    flat = s.reshape(-1, rows, nkb)
+    out = np.empty((flat.shape[0], ng, rows), dtype=np.int32)
+    for i in range(flat.shape[0]):
+        src = np.ascontiguousarray(flat[i])
+        dst = np.empty((ng, rows), dtype=np.int32)
+        if _load().dgo_pack_ue8m0(_ptr(src), rows, nkb, _ptr(dst)):
+            raise ValueError("pack_ue8m0: a scale is not a power of two in UE8M0 range")
+        out[i] = dst
+    return out.reshape(*lead, ng, rows)
+
+
+def unpack_ue8m0(packed, nkb: int):
+    """Inverse of pack_ue8m0: [..., ceil(nkb/4), rows] -> [..., rows, nkb]."""
+    packed = np.ascontiguousarray(packed, dtype=np.int32)
+    *lead, ng, rows = packed.shape
+    assert ng == (nkb + 3) // 4
+    flat = packed.reshape(-1, ng, rows)
+    out = np.empty((flat.shape[0], rows, nkb), dtype=np.float32)
+    for i in range(flat.shape[0]):
+        dst = np.empty((rows, nkb), dtype=np.float32)
+        _load().dgo_unpack_ue8m0(_ptr(np.ascontiguousarray(flat[i])), rows, nkb, _ptr(dst))
+        out[i] = dst
+    return out.reshape(*lead, rows, nkb)
+
+
+def gemm_nt_ue8m0(A, sfa, B, sfb, want_f64: bool = True):
+    """Dense GEMM with packed UE8M0 scales: sfa [ceil(K/512)][M],
+    sfb [ceil(K/512)][ceil(N/128)] (pack_ue8m0 of the logical scales)."""
+    nkb = np.asarray(A).shape[-1] // BLOCK
+    return gemm_nt(A, unpack_ue8m0(sfa, nkb), B, unpack_ue8m0(sfb, nkb), want_f64)
+
+
+def grouped_contiguous_ue8m0(A, sfa, B, sfb, m_indices, D16_init, want_f64=False):
+    """grouped_contiguous with packed UE8M0 scales: sfa [ceil(K/512)][M_total],
+    sfb [G][ceil(K/512)][ceil(N/128)]."""
+    nkb = np.asarray(A).shape[-1] // BLOCK
+    return grouped_contiguous(A, unpack_ue8m0(sfa, nkb), B, unpack_ue8m0(sfb, nkb), m_indices,
+                              D16_init, want_f64)
+
+
+def grouped_masked_ue8m0(A, sfa, B, sfb, masked_m, D16_init, want_f64=False):
+    """grouped_masked with packed UE8M0 scales: sfa [G][ceil(K/512)][max_m],
+    sfb [G][ceil(K/512)][ceil(N/128)]."""
+    nkb = np.asarray(A).shape[-1] // BLOCK
+    return grouped_masked(A, unpack_ue8m0(sfa, nkb), B, unpack_ue8m0(sfb, nkb), masked_m,
+                          D16_init, want_f64)

@@ -444,3 +444,98 @@ int dgo_num_threads(void)
     return 1;
 #endif
 }
+
+/* ---------------------------------------------------------- UE8M0 scales
+ *
+ * The block-scaled mode of the SM100 path takes its scales as UE8M0 (an
+ * unsigned 8-bit biased exponent e, value 2^(e-127), e = 255 is NaN), four
+ * of them packed into one 32-bit integer, in a transposed (MN-major) layout
+ * (hada.io page, section "Giao dien GEMM va rang buoc layout": the SM100
+ * scaling factors are packed UE8M0, four to an int, and the LHS scales are
+ * TMA-aligned and transposed).
+ *
+ * Readings where the pages are silent:
+ *  - byte j (bits 8j .. 8j+7) of the integer for row r and group g holds the
+ *    scale of K block 4g + j; bytes past the last K block hold 127 (value 1);
+ *  - the packed array is [ceil(nkb/4)][rows] (MN-major);
+ *  - a UE8M0 quantiser picks, per block, the smallest power of two s with
+ *    amax / s <= 448, i.e. s = 2^ceil(log2(amax / 448)), and the data is
+ *    quantised with that s.
+ * The GEMM itself is unchanged: with the scales decoded, dgo_gemm_nt and the
+ * grouped forms above compute the block-scaled result.
+ */
+
+/* UE8M0 code -> value: 2^(e-127); e = 255 is NaN. */
+double dgo_ue8m0_value(uint8_t e)
+{
+    if (e == 255)
+        return NAN;
+    return ldexp(1.0, (int)e - 127);
+}
+
+/* Exact encoding: s must be a power of two in [2^-127, 2^127]; returns its
+ * code, or -1 for anything else (zero, negative, not a power of two, out of
+ * range, inf, NaN). */
+int dgo_ue8m0_from_scale(double s)
+{
+    if (!(s > 0.0) || isinf(s))
+        return -1;
+    int ex;
+    double m = frexp(s, &ex); /* s = m * 2^ex, 0.5 <= m < 1 */
+    if (m != 0.5)
+        return -1;
+    int e = ex - 1 + 127;
+    if (e < 0 || e > 254)
+        return -1;
+    return e;
+}
+
+/* The smallest power of two >= x, for finite x > 0. */
+double dgo_ue8m0_ceil_pow2(double x)
+{
+    int ex;
+    double m = frexp(x, &ex);
+    return m == 0.5 ? x : ldexp(1.0, ex);
+}
+
+/* s: [rows][nkb] fp32 scales (powers of two) -> out: [ceil(nkb/4)][rows]
+ * packed codes.  Returns 1 (and leaves out partly written) if a scale is not
+ * representable. */
+int dgo_pack_ue8m0(const float *s, int rows, int nkb, int32_t *out)
+{
+    if (rows < 0 || nkb < 1)
+        return 1;
+    int ngroups = (nkb + 3) / 4;
+    for (int g = 0; g < ngroups; ++g) {
+        for (int r = 0; r < rows; ++r) {
+            uint32_t word = 0;
+            for (int j = 0; j < 4; ++j) {
+                int kb = 4 * g + j;
+                int code = 127;
+                if (kb < nkb) {
+                    code = dgo_ue8m0_from_scale((double)s[(int64_t)r * nkb + kb]);
+                    if (code < 0)
+                        return 1;
+                }
+                word |= (uint32_t)code << (8 * j);
+            }
+            out[(int64_t)g * rows + r] = (int32_t)word;
+        }
+    }
+    return 0;
+}
+
+/* Inverse of dgo_pack_ue8m0: in [ceil(nkb/4)][rows] -> s [rows][nkb]. */
+int dgo_unpack_ue8m0(const int32_t *in, int rows, int nkb, float *s)
+{
+    if (rows < 0 || nkb < 1)
+        return 1;
+    for (int r = 0; r < rows; ++r) {
+        for (int kb = 0; kb < nkb; ++kb) {
+            uint32_t word = (uint32_t)in[(int64_t)(kb / 4) * rows + r];
+            uint8_t code = (uint8_t)((word >> (8 * (kb % 4))) & 0xFFu);
+            s[(int64_t)r * nkb + kb] = (float)dgo_ue8m0_value(code);
+        }
+    }
+    return 0;
+}

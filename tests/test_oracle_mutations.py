@@ -3,7 +3,8 @@
 Each case plants one mistake in a temporary copy of oracle/dg_oracle.c -- a
 wrong weight-block index, a transposed operand stride, a dropped K block, a
 lost accumulation, an exponent bias off by one, truncation instead of
-round-to-nearest-even -- builds it with gcc, and checks that at least one of
+round-to-nearest-even, a UE8M0 bias, rounding direction or byte order --
+builds it with gcc, and checks that at least one of
 the independent pins (torch's casts, float64 matmul of the dequantised
 inputs) rejects it.  The committed oracle itself is never modified."""
 import ctypes
@@ -44,6 +45,15 @@ MUTATIONS = {
     "accumulator C dropped from D = C + A.B^T": (
         "            double v = (double)C[(int64_t)m * N + n] +\n                       dgo_element(",
         "            double v = 0.0 * (double)C[(int64_t)m * N + n] +\n                       dgo_element("),
+    "UE8M0 exponent bias 128 instead of 127": (
+        "    return ldexp(1.0, (int)e - 127);",
+        "    return ldexp(1.0, (int)e - 128);"),
+    "UE8M0 scale rounded down instead of up": (
+        "    return m == 0.5 ? x : ldexp(1.0, ex);",
+        "    return m == 0.5 ? x : ldexp(1.0, ex - 1);"),
+    "UE8M0 packing byte order reversed": (
+        "                word |= (uint32_t)code << (8 * j);",
+        "                word |= (uint32_t)code << (8 * (3 - j));"),
 }
 
 
@@ -65,6 +75,12 @@ def _build_variant(tmp_path, old, new):
     lib.dgo_gemm_nt_acc.restype = I
     lib.dgo_k_grouped_tn.argtypes = [P, P, P, P, P, I, I, I, I, P, P]
     lib.dgo_k_grouped_tn.restype = I
+    lib.dgo_ue8m0_value.restype = ctypes.c_double
+    lib.dgo_ue8m0_value.argtypes = [ctypes.c_uint8]
+    lib.dgo_ue8m0_ceil_pow2.restype = ctypes.c_double
+    lib.dgo_ue8m0_ceil_pow2.argtypes = [ctypes.c_double]
+    lib.dgo_pack_ue8m0.restype = I
+    lib.dgo_pack_ue8m0.argtypes = [P, I, I, P]
     return lib
 
 
@@ -131,6 +147,25 @@ def _pins_pass(lib) -> bool:
         bound = np.abs(ka[off[g]:off[g + 1]]).T @ np.abs(kb[off[g]:off[g + 1]])
         if not np.all(np.abs(k64[g] - ref) <= 1e-12 * bound + 1e-300):
             return False
+    # UE8M0: code values, the rounding rule against a doubling search, and
+    # the hand-worked packing example
+    if any(lib.dgo_ue8m0_value(e) != 2.0 ** (e - 127) for e in range(255)):
+        return False
+    for x in [3.0, 0.3, 1.0, 1e-9, 5e6, 2.0 ** -20 * 1.0000001]:
+        s = 1.0
+        while s < x:
+            s *= 2.0
+        while s / 2.0 >= x:
+            s /= 2.0
+        if lib.dgo_ue8m0_ceil_pow2(x) != s:
+            return False
+    sc = np.array([[1, 2, 0.5, 8, 32], [0.25, 1, 1, 1, 1]], np.float32)
+    words = np.empty((2, 2), np.int32)
+    if lib.dgo_pack_ue8m0(_ptr(sc), 2, 5, _ptr(words)) != 0:
+        return False
+    want = np.array([[0x827E807F, 0x7F7F7F7D], [0x7F7F7F84, 0x7F7F7F7F]], dtype=np.uint32)
+    if not np.array_equal(words.view(np.uint32), want):
+        return False
     return True
 
 
