@@ -72,8 +72,10 @@ typedef enum {
     DG_ERR_CUDA = 4,           /* a CUDA runtime or driver call failed       */
     DG_ERR_TIMEOUT = 5,        /* device: a pipeline wait ran out of time    */
     DG_ERR_BAD_GROUP_DATA = 6, /* device: m_indices / masked_m out of range  */
-    DG_ERR_WORKSPACE_LIMIT = 7 /* problem too large for the fixed scratch of
-                                  dg_fp8_gemm_nt_noalloc                    */
+    DG_ERR_WORKSPACE_LIMIT = 7, /* problem too large for the fixed scratch of
+                                   dg_fp8_gemm_nt_noalloc                    */
+    DG_ERR_BAD_SCALE = 8        /* device: dg_transform_sf_ue8m0 met a scale
+                                   that is not a UE8M0 power of two          */
 } dg_status_t;
 
 /*
@@ -229,6 +231,70 @@ dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, const void *B
                                    const float *sB, void *D, int M, int N, int K,
                                    cudaStream_t stream);
 
+/*
+ * UE8M0 block-scaled mode (a separately declared mode of the same GEMM).
+ *
+ * The SM100 path of the pages takes its scaling factors as packed UE8M0,
+ * four to an int (hada.io page, section "Giao dien GEMM va rang buoc
+ * layout").  UE8M0 is an unsigned 8-bit biased exponent: code e is the scale
+ * 2^(e-127) (e = 255 is NaN), so every scale is a power of two.  The tensor
+ * core then applies the scales itself (tcgen05.mma kind::mxf8f6f4 with block
+ * scaling) and accumulates the whole K range in fp32:
+ *
+ *   D[m,n] = bf16( sum_kb 2^(ea[m,kb]-127) * 2^(eb[n/128,kb]-127)
+ *                         * sum_{k in block kb} A[m,k]*B[n,k] )
+ *
+ * which is the fine-grained-scaled result for those (power-of-two) scales,
+ * up to the order of the fp32 additions.  Quantising with power-of-two
+ * scales (the smallest 2^k >= amax/448 per block) is the caller's part, as
+ * the cast to FP8 is in the fp32-scale mode.
+ *
+ * Packed scale layouts (int32 words; byte j = bits 8j..8j+7 of the word for
+ * K-block group g holds K block 4g+j, bytes past the last K block are
+ * ignored; ng = ceil(K/512)):
+ *   sfa : dense/contiguous [ng][M_pad], masked [G][ng][max_m_pad], with
+ *         X_pad = dg_get_tma_aligned_size(X, 4) (transposed, TMA-aligned,
+ *         16-byte aligned base); pad entries unread
+ *   sfb : [G][ng][ceil(N/128)] (G = 1 for dense), one word per 128x128
+ *         weight block, 4-byte aligned
+ * dg_transform_sf_ue8m0 builds both from the fp32 scale layouts.  A, B, D,
+ * m_indices, masked_m, the validation rules and the device status behaviour
+ * are those of dg_fp8_gemm_nt, dg_fp8_grouped_gemm_contiguous and
+ * dg_fp8_grouped_gemm_masked.  These calls run one-CTA tiles (128 x BN, BN
+ * in {128, 160, 192, 224}) and allocate nothing.
+ */
+dg_status_t dg_fp8_gemm_nt_ue8m0(const void *A, const int32_t *sfa, const void *B,
+                                 const int32_t *sfb, void *D, int M, int N, int K,
+                                 cudaStream_t stream);
+dg_status_t dg_fp8_grouped_gemm_contiguous_ue8m0(const void *A, const int32_t *sfa,
+                                                 const void *B, const int32_t *sfb, void *D,
+                                                 const int32_t *m_indices, int M_total, int N,
+                                                 int K, int num_groups, cudaStream_t stream);
+dg_status_t dg_fp8_grouped_gemm_masked_ue8m0(const void *A, const int32_t *sfa, const void *B,
+                                             const int32_t *sfb, void *D,
+                                             const int32_t *masked_m, int num_groups,
+                                             int max_m, int N, int K, int expected_m,
+                                             cudaStream_t stream);
+
+/*
+ * Packs fp32 scales into the UE8M0 words above (the pages'
+ * transform_sf_into_required_layout, hada.io page, section "Tien ich va bien
+ * moi truong", for the SM100 format).  K is the GEMM's K (nkb = K/128 scales
+ * per row); batch is 1, or G for per-group scale arrays.
+ *   mn_major = 1: sf [batch][nkb][rows_pad] (the LHS-scale layout, rows_pad =
+ *                 dg_get_tma_aligned_size(rows, 4)) -> out [batch][ng][rows_pad]
+ *   mn_major = 0: sf [batch][rows][nkb] (the weight-scale layout, rows =
+ *                 ceil(N/128)) -> out [batch][ng][rows]
+ * Each scale must be a power of two in [2^-127, 2^127] (an fp32 value with a
+ * zero mantissa, or the subnormal 2^-127); its code is exact.  Any other
+ * value is packed as 255 (NaN, so the GEMM result shows it) and raises
+ * DG_ERR_BAD_SCALE in the device status word.  Pad rows and bytes past the
+ * last K block become 127 (scale 1).  Device pointers, asynchronous on
+ * `stream`; rows == 0 is a no-op.
+ */
+dg_status_t dg_transform_sf_ue8m0(const float *sf, int32_t *out, int rows, int K, int batch,
+                                  int mn_major, cudaStream_t stream);
+
 /* Row alignment of each group's segment in the contiguous layout (128). */
 int dg_get_mk_alignment_for_contiguous_layout(void);
 
@@ -281,8 +347,9 @@ dg_status_t dg_get_device_status(cudaStream_t stream);
 dg_status_t dg_get_device_status_detail(cudaStream_t stream, uint32_t *word);
 
 /* Describes the kernel configuration the library would launch for a problem
- * (layout 0 = dense, 1 = contiguous, 2 = masked; for masked, M = expected_m
- * and groups = G) into buf (NUL-terminated, truncated to len).  Returns the
+ * (layout 0 = dense, 1 = contiguous, 2 = masked, and 3, 4, 5 for the same
+ * layouts in the UE8M0 block-scaled mode; for masked, M = expected_m and
+ * groups = G) into buf (NUL-terminated, truncated to len).  Returns the
  * number of characters it wanted to write, or -1 on bad arguments. */
 int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf,
                        int len);

@@ -15,6 +15,12 @@ Layouts (row-major, packed):
 with X_pad = get_tma_aligned_size(X, 4) (the transposed, TMA-aligned LHS
 scale layout of the DeepGEMM pages, hada.io summary, section "Giao dien GEMM
 va rang buoc layout").
+
+UE8M0 block-scaled mode (``*_ue8m0``): the same A, B, D and group metadata
+with packed int32 scale words, four K blocks per word (ng = ceil(K/512)):
+sfa [ng, M_pad] (masked: [G, ng, max_m_pad]) and sfb [G, ng, ceil(N/128)]
+(dense: [1, ng, ceil(N/128)] or [ng, ceil(N/128)]); dg_transform_sf_ue8m0
+packs them from the fp32 layouts above.
 """
 from __future__ import annotations
 
@@ -30,7 +36,7 @@ DG_OK = 0
 STATUS_NAMES = {
     0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_UNSUPPORTED", 3: "DG_ERR_ALIGNMENT",
     4: "DG_ERR_CUDA", 5: "DG_ERR_TIMEOUT", 6: "DG_ERR_BAD_GROUP_DATA",
-    7: "DG_ERR_WORKSPACE_LIMIT",
+    7: "DG_ERR_WORKSPACE_LIMIT", 8: "DG_ERR_BAD_SCALE",
 }
 LAYOUT_DENSE, LAYOUT_CONTIGUOUS, LAYOUT_MASKED = 0, 1, 2
 
@@ -47,6 +53,10 @@ _SIGNATURES = {
     "dg_fp8_gemm_nt_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "dg_fp8_grouped_gemm_contiguous": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "dg_fp8_grouped_gemm_masked": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "dg_fp8_gemm_nt_ue8m0": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "dg_fp8_grouped_gemm_contiguous_ue8m0": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "dg_fp8_grouped_gemm_masked_ue8m0": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "dg_transform_sf_ue8m0": (_I, [_P, _P, _I, _I, _I, _I, _P]),
     "dg_get_mk_alignment_for_contiguous_layout": (_I, []),
     "dg_get_tma_aligned_size": (_I, [_I, _I]),
     "dg_set_num_sms": (_I, [_I]),
@@ -368,3 +378,119 @@ def dg_fp8_grouped_gemm_masked(A, sA, B, sB, D, masked_m, expected_m: int = 0, s
     st = load_library().dg_fp8_grouped_gemm_masked(pa, psa, pb, psb, pd, pm, G, max_m, N, K,
                                                    expected_m, _stream_handle(stream, A.device))
     _check("dg_fp8_grouped_gemm_masked", st)
+
+
+# ------------------------------------------------------- UE8M0 block-scaled
+
+def _ng(K: int) -> int:
+    return (K // 128 + 3) // 4
+
+
+def dg_transform_sf_ue8m0(sf, rows: int, mn_major: bool = True, out=None, stream=None):
+    """Packs fp32 power-of-two scales into UE8M0 words (four K blocks per
+    int32).  mn_major: sf [..., K/128, rows_pad] (the LHS layout, rows_pad =
+    get_tma_aligned_size(rows, 4)) -> out [..., ceil(K/512), rows_pad]; else
+    sf [..., rows, K/128] (the weight layout) -> out [..., ceil(K/512), rows].
+    Returns out (allocated when None).  A scale that is not a power of two is
+    packed as NaN and flagged DG_ERR_BAD_SCALE in the device status word."""
+    if not isinstance(sf, torch.Tensor) or not sf.is_cuda or sf.dtype != torch.float32:
+        raise ValueError("sf must be a float32 CUDA tensor")
+    if not sf.is_contiguous() or sf.dim() < 2:
+        raise ValueError("sf must be contiguous with at least 2 dims")
+    batch = 1
+    for d in sf.shape[:-2]:
+        batch *= d
+    if mn_major:
+        nkb, ld = sf.shape[-2], sf.shape[-1]
+        if ld != get_tma_aligned_size(rows, 4):
+            raise ValueError(f"sf must be [..., K/128, {get_tma_aligned_size(rows, 4)}]")
+    else:
+        if sf.shape[-2] != rows:
+            raise ValueError(f"sf must be [..., {rows}, K/128]")
+        nkb, ld = sf.shape[-1], rows
+    K = nkb * 128
+    out_shape = (*sf.shape[:-2], _ng(K), ld)
+    if out is None:
+        out = torch.empty(out_shape, dtype=torch.int32, device=sf.device)
+    po = _dev(out, "out", _I32, len(out_shape))
+    if tuple(out.shape) != tuple(out_shape):
+        raise ValueError(f"out must be {out_shape}")
+    st = load_library().dg_transform_sf_ue8m0(sf.data_ptr(), po, rows, K, batch, 1 if mn_major else 0,
+                                              _stream_handle(stream, sf.device))
+    _check("dg_transform_sf_ue8m0", st)
+    return out
+
+
+def dg_fp8_gemm_nt_ue8m0(A, sfa, B, sfb, D, stream=None) -> None:
+    """Dense NT GEMM in the UE8M0 block-scaled mode: sfa [ng, M_pad],
+    sfb [ng, ceil(N/128)] (or [1, ng, ceil(N/128)]) packed int32."""
+    pa = _dev(A, "A", _FP8, 2)
+    M, K = A.shape
+    pb = _dev(B, "B", _FP8, 2)
+    if B.shape[1] != K:
+        raise ValueError("B must be [N, K]")
+    N = B.shape[0]
+    psa = _dev(sfa, "sfa", _I32, 2)
+    if tuple(sfa.shape) != (_ng(K), get_tma_aligned_size(M, 4)):
+        raise ValueError(f"sfa must be [ceil(K/512), M_pad] = {(_ng(K), get_tma_aligned_size(M, 4))}")
+    psb = _dev(sfb, "sfb", _I32, sfb.dim() if isinstance(sfb, torch.Tensor) and sfb.dim() in (2, 3) else 2)
+    if tuple(sfb.shape)[-2:] != (_ng(K), (N + 127) // 128) or (sfb.dim() == 3 and sfb.shape[0] != 1):
+        raise ValueError("sfb must be [ceil(K/512), ceil(N/128)]")
+    pd = _dev(D, "D", _BF16, 2)
+    if tuple(D.shape) != (M, N):
+        raise ValueError("D must be [M, N]")
+    st = load_library().dg_fp8_gemm_nt_ue8m0(pa, psa, pb, psb, pd, M, N, K, _stream_handle(stream, A.device))
+    _check("dg_fp8_gemm_nt_ue8m0", st)
+
+
+def dg_fp8_grouped_gemm_contiguous_ue8m0(A, sfa, B, sfb, D, m_indices, stream=None) -> None:
+    """Contiguous grouped GEMM in the UE8M0 mode: sfa [ng, M_total_pad],
+    sfb [G, ng, ceil(N/128)]."""
+    pa = _dev(A, "A", _FP8, 2)
+    M, K = A.shape
+    pb = _dev(B, "B", _FP8, 3)
+    G, N, Kb = B.shape
+    if Kb != K:
+        raise ValueError("B must be [G, N, K]")
+    psa = _dev(sfa, "sfa", _I32, 2)
+    if tuple(sfa.shape) != (_ng(K), get_tma_aligned_size(M, 4)):
+        raise ValueError("sfa must be [ceil(K/512), M_pad]")
+    psb = _dev(sfb, "sfb", _I32, 3)
+    if tuple(sfb.shape) != (G, _ng(K), (N + 127) // 128):
+        raise ValueError("sfb must be [G, ceil(K/512), ceil(N/128)]")
+    pd = _dev(D, "D", _BF16, 2)
+    if tuple(D.shape) != (M, N):
+        raise ValueError("D must be [M_total, N]")
+    pm = _dev(m_indices, "m_indices", _I32, 1)
+    if m_indices.shape[0] != M:
+        raise ValueError("m_indices must be [M_total]")
+    st = load_library().dg_fp8_grouped_gemm_contiguous_ue8m0(pa, psa, pb, psb, pd, pm, M, N, K, G,
+                                                             _stream_handle(stream, A.device))
+    _check("dg_fp8_grouped_gemm_contiguous_ue8m0", st)
+
+
+def dg_fp8_grouped_gemm_masked_ue8m0(A, sfa, B, sfb, D, masked_m, expected_m: int = 0,
+                                     stream=None) -> None:
+    """Masked grouped GEMM in the UE8M0 mode: sfa [G, ng, max_m_pad],
+    sfb [G, ng, ceil(N/128)]."""
+    pa = _dev(A, "A", _FP8, 3)
+    G, max_m, K = A.shape
+    pb = _dev(B, "B", _FP8, 3)
+    if B.shape[0] != G or B.shape[2] != K:
+        raise ValueError("B must be [G, N, K]")
+    N = B.shape[1]
+    psa = _dev(sfa, "sfa", _I32, 3)
+    if tuple(sfa.shape) != (G, _ng(K), get_tma_aligned_size(max_m, 4)):
+        raise ValueError("sfa must be [G, ceil(K/512), max_m_pad]")
+    psb = _dev(sfb, "sfb", _I32, 3)
+    if tuple(sfb.shape) != (G, _ng(K), (N + 127) // 128):
+        raise ValueError("sfb must be [G, ceil(K/512), ceil(N/128)]")
+    pd = _dev(D, "D", _BF16, 3)
+    if tuple(D.shape) != (G, max_m, N):
+        raise ValueError("D must be [G, max_m, N]")
+    pm = _dev(masked_m, "masked_m", _I32, 1)
+    if masked_m.shape[0] != G:
+        raise ValueError("masked_m must be [G]")
+    st = load_library().dg_fp8_grouped_gemm_masked_ue8m0(pa, psa, pb, psb, pd, pm, G, max_m, N, K,
+                                                         expected_m, _stream_handle(stream, A.device))
+    _check("dg_fp8_grouped_gemm_masked_ue8m0", st)

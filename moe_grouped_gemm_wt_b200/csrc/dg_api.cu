@@ -1,7 +1,8 @@
 // dg_api.cu -- host side of the C ABI declared in include/dg_b200.h:
 // argument validation, tile-shape choice, TMA descriptor encoding and kernel
 // launch.  All arithmetic of the GEMM runs in fp8_gemm_kernel.cuh (one CTA
-// per tile) and fp8_gemm_pair_kernel.cuh (a CTA pair per 256-row tile).
+// per tile), fp8_gemm_pair_kernel.cuh (a CTA pair per 256-row tile) and
+// fp8_gemm_bs_kernel.cuh (the UE8M0 block-scaled mode and its scale packing).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -12,6 +13,7 @@
 #include <mutex>
 
 #include "../../include/dg_b200.h"
+#include "fp8_gemm_bs_kernel.cuh"
 #include "fp8_gemm_kernel.cuh"
 #include "fp8_gemm_pair_kernel.cuh"
 
@@ -639,6 +641,132 @@ dg_status_t dense_gemm(const void *A, const float *sA, const void *B, const floa
     return dispatch<dg::kDense>(plan, A, am, B, bn, p, sms, stream);
 }
 
+// ------------------------------------------------ UE8M0 block-scaled mode
+
+// Tile shapes of the block-scaled kernel.  The tensor core applies the
+// scales, so a tile's time is its MMA time (proportional to BN) plus a fixed
+// fill/epilogue part; the planner takes the fewest waves x (BN + 48).
+struct BsChoice {
+    int bn, stages, ks;
+};
+constexpr BsChoice kBsChoices[] = {{128, 3, 2}, {160, 2, 2}, {192, 2, 2}, {224, 2, 2}};
+
+BsChoice choose_bs(int64_t m_blocks, int N, int sms)
+{
+    BsChoice best = kBsChoices[0];
+    double best_cost = 1e300;
+    for (const BsChoice &c : kBsChoices) {
+        if (forced_block_n() > 0 && c.bn != forced_block_n())
+            continue;
+        const int64_t tiles = m_blocks * ((N + c.bn - 1) / c.bn);
+        const int64_t waves = (tiles + sms - 1) / sms;
+        const double cost = static_cast<double>(waves) * (c.bn + 48);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = c;
+        }
+    }
+    return best;
+}
+
+template <int BN, int STAGES, int KS, int LAYOUT>
+dg_status_t launch_bs(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows, const GemmParams &p,
+                      int grid, cudaStream_t stream)
+{
+    using Cfg = dg::BsConfig<BN, STAGES, KS>;
+    CUtensorMap ta, tb, td64, tdrem;
+    if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
+        !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, BN, KS))
+        return DG_ERR_CUDA;
+    if (!make_tmap_bf16(&td64, p.D, static_cast<uint64_t>(p.N), a_rows, 64, dg::kBM,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return DG_ERR_CUDA;
+    if (Cfg::EPI_REM > 0) {
+        if (!make_tmap_bf16(&tdrem, p.D, static_cast<uint64_t>(p.N), a_rows, Cfg::EPI_REM, dg::kBM,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+            return DG_ERR_CUDA;
+    } else {
+        tdrem = td64;
+    }
+    auto kern = dg::fp8_gemm_bs_kernel<BN, STAGES, KS, LAYOUT>;
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices)
+        return DG_ERR_CUDA;
+    if (!attr_set[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) !=
+            cudaSuccess)
+            return DG_ERR_CUDA;
+        attr_set[dev].store(true);
+    }
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, td64, tdrem, p);
+    if (cudaPeekAtLastError() != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DG_ERR_CUDA;
+    }
+    return DG_OK;
+}
+
+template <int LAYOUT>
+dg_status_t dispatch_bs(const BsChoice &c, const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
+                        GemmParams p, int sms, cudaStream_t stream)
+{
+    p.num_nb = (p.N + c.bn - 1) / c.bn;
+    p.ksplit = 1;
+    p.kb_per_split = p.num_kb;
+    const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
+    int grid = sms;
+    if (LAYOUT != dg::kMasked)
+        grid = static_cast<int>(tiles < sms ? tiles : sms);
+    if (grid <= 0)
+        return DG_OK;
+#define DG_BS_CASE(BN_, ST_, KS_)                                                                   \
+    if (c.bn == BN_ && c.stages == ST_ && c.ks == KS_)                                               \
+        return launch_bs<BN_, ST_, KS_, LAYOUT>(A, a_rows, B, b_rows, p, grid, stream);
+    DG_BS_CASE(128, 3, 2)
+    DG_BS_CASE(160, 2, 2)
+    DG_BS_CASE(192, 2, 2)
+    DG_BS_CASE(224, 2, 2)
+#undef DG_BS_CASE
+    return DG_ERR_UNSUPPORTED;
+}
+
+dg_status_t check_bs(const void *A, const int32_t *sfa, const void *B, const int32_t *sfb, const void *D,
+                     int N, int K)
+{
+    if (!A || !sfa || !B || !sfb || !D)
+        return DG_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0)
+        return DG_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N % 16 != 0)
+        return DG_ERR_UNSUPPORTED;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16) || !aligned(sfa, 16) || !aligned(sfb, 4))
+        return DG_ERR_ALIGNMENT;
+    return DG_OK;
+}
+
+// Parameters shared by the three layouts of the block-scaled mode.
+GemmParams bs_params(const int32_t *sfa, const int32_t *sfb, void *D, int M, int N, int K, int G)
+{
+    GemmParams p{};
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.D = static_cast<__nv_bfloat16 *>(D);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = G;
+    p.sfa_ld = dg_get_tma_aligned_size(M, 4);
+    p.num_kb = K / 128;
+    p.num_kg = (p.num_kb + 3) / 4;
+    p.nbn = (N + 127) / 128;
+    p.num_mb = (M + 127) / 128;
+    p.raster = choose_raster(p.num_mb);
+    p.timeout_ns = g_timeout_ns.load();
+    p.stall_injection = g_stall_injection.load();
+    return p;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -864,6 +992,117 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const voi
                                  static_cast<uint64_t>(num_groups) * N, p, sms, stream);
 }
 
+dg_status_t dg_fp8_gemm_nt_ue8m0(const void *A, const int32_t *sfa, const void *B, const int32_t *sfb,
+                                 void *D, int M, int N, int K, cudaStream_t stream)
+{
+    if (M < 0)
+        return DG_ERR_INVALID_ARG;
+    dg_status_t st = check_bs(A, sfa, B, sfb, D, N, K);
+    if (st != DG_OK)
+        return st;
+    if (M == 0)
+        return DG_OK;
+    const int sms = effective_sms(current_device());
+    if (sms <= 0)
+        return DG_ERR_CUDA;
+    GemmParams p = bs_params(sfa, sfb, D, M, N, K, 1);
+    const BsChoice c = choose_bs(p.num_mb, N, sms);
+    if (print_configs())
+        std::fprintf(stderr, "[dg] dense ue8m0 M=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n", M, N,
+                     K, c.bn, c.stages, c.ks, sms);
+    return dispatch_bs<dg::kDense>(c, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), p, sms,
+                                   stream);
+}
+
+dg_status_t dg_fp8_grouped_gemm_contiguous_ue8m0(const void *A, const int32_t *sfa, const void *B,
+                                                 const int32_t *sfb, void *D, const int32_t *m_indices,
+                                                 int M_total, int N, int K, int num_groups,
+                                                 cudaStream_t stream)
+{
+    if (M_total < 0 || num_groups <= 0 || !m_indices)
+        return DG_ERR_INVALID_ARG;
+    dg_status_t st = check_bs(A, sfa, B, sfb, D, N, K);
+    if (st != DG_OK)
+        return st;
+    if (M_total % 128 != 0)
+        return DG_ERR_UNSUPPORTED;
+    if (!aligned(m_indices, 4))
+        return DG_ERR_ALIGNMENT;
+    if (M_total == 0)
+        return DG_OK;
+    if (static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF)
+        return DG_ERR_UNSUPPORTED;
+    const int sms = effective_sms(current_device());
+    if (sms <= 0)
+        return DG_ERR_CUDA;
+    GemmParams p = bs_params(sfa, sfb, D, M_total, N, K, num_groups);
+    p.m_indices = m_indices;
+    const BsChoice c = choose_bs(p.num_mb, N, sms);
+    if (print_configs())
+        std::fprintf(stderr, "[dg] contiguous ue8m0 M=%d N=%d K=%d G=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
+                     M_total, N, K, num_groups, c.bn, c.stages, c.ks, sms);
+    return dispatch_bs<dg::kContiguous>(c, A, static_cast<uint64_t>(M_total), B,
+                                        static_cast<uint64_t>(num_groups) * N, p, sms, stream);
+}
+
+dg_status_t dg_fp8_grouped_gemm_masked_ue8m0(const void *A, const int32_t *sfa, const void *B,
+                                             const int32_t *sfb, void *D, const int32_t *masked_m,
+                                             int num_groups, int max_m, int N, int K, int expected_m,
+                                             cudaStream_t stream)
+{
+    if (num_groups <= 0 || max_m < 0 || expected_m < 0 || !masked_m)
+        return DG_ERR_INVALID_ARG;
+    dg_status_t st = check_bs(A, sfa, B, sfb, D, N, K);
+    if (st != DG_OK)
+        return st;
+    if (!aligned(masked_m, 4))
+        return DG_ERR_ALIGNMENT;
+    if (max_m == 0)
+        return DG_OK;
+    if (static_cast<int64_t>(num_groups) * max_m > 0x7FFFFFFF ||
+        static_cast<int64_t>(num_groups) * N > 0x7FFFFFFF)
+        return DG_ERR_UNSUPPORTED;
+    const int sms = effective_sms(current_device());
+    if (sms <= 0)
+        return DG_ERR_CUDA;
+    GemmParams p = bs_params(sfa, sfb, D, max_m, N, K, num_groups);
+    p.masked_m = masked_m;
+    p.raster = 1;
+    const int em = (expected_m > 0 && expected_m < max_m) ? expected_m : max_m;
+    const BsChoice c = choose_bs(static_cast<int64_t>(num_groups) * ((em + 127) / 128), N, sms);
+    if (print_configs())
+        std::fprintf(stderr,
+                     "[dg] masked ue8m0 G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
+                     num_groups, max_m, em, N, K, c.bn, c.stages, c.ks, sms);
+    return dispatch_bs<dg::kMasked>(c, A, static_cast<uint64_t>(num_groups) * max_m, B,
+                                    static_cast<uint64_t>(num_groups) * N, p, sms, stream);
+}
+
+dg_status_t dg_transform_sf_ue8m0(const float *sf, int32_t *out, int rows, int K, int batch, int mn_major,
+                                  cudaStream_t stream)
+{
+    if (!sf || !out || rows < 0 || K <= 0 || batch <= 0 || (mn_major != 0 && mn_major != 1))
+        return DG_ERR_INVALID_ARG;
+    if (K % 128 != 0)
+        return DG_ERR_UNSUPPORTED;
+    if (!aligned(sf, 4) || !aligned(out, 4))
+        return DG_ERR_ALIGNMENT;
+    if (rows == 0)
+        return DG_OK;
+    const int out_ld = mn_major ? dg_get_tma_aligned_size(rows, 4) : rows;
+    const int nkb = K / 128;
+    const int64_t total = static_cast<int64_t>(batch) * ((nkb + 3) / 4) * out_ld;
+    const int threads = 256;
+    const int64_t want = (total + threads - 1) / threads;
+    const int blocks = static_cast<int>(want < 4096 ? want : 4096);
+    dg::transform_sf_ue8m0_kernel<<<blocks, threads, 0, stream>>>(sf, out, rows, out_ld, nkb, batch, mn_major);
+    if (cudaPeekAtLastError() != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DG_ERR_CUDA;
+    }
+    return DG_OK;
+}
+
 int dg_get_mk_alignment_for_contiguous_layout(void) { return 128; }
 
 int dg_get_tma_aligned_size(int x, int elem_bytes)
@@ -934,13 +1173,22 @@ dg_status_t dg_get_device_status(cudaStream_t stream)
 
 int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, int len)
 {
-    if (layout < 0 || layout > 2 || M < 0 || N <= 0 || K <= 0 || groups <= 0 || (len > 0 && !buf))
+    if (layout < 0 || layout > 5 || M < 0 || N <= 0 || K <= 0 || groups <= 0 || (len > 0 && !buf))
         return -1;
     // Without a device (host-only use) the SM cap alone decides, else 148.
     const int dev = current_device();
     int sms = effective_sms(dev);
     if (sms <= 0)
         sms = g_num_sms_cap.load() > 0 ? g_num_sms_cap.load() : 148;
+    if (layout >= 3) {
+        // the UE8M0 block-scaled mode (one-CTA tiles, no K split)
+        const int64_t mb = static_cast<int64_t>((M + 127) / 128) * (layout == 5 ? groups : 1);
+        const BsChoice c = choose_bs(mb, N, sms);
+        return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
+                             "layout=%d BM=128 BN=%d BK=128 stages=%d ks=%d ksplit=1 pair=0 wg=1 sms=%d m_blocks=%lld n_blocks=%d ue8m0=1",
+                             layout, c.bn, c.stages, c.ks, sms, static_cast<long long>(mb),
+                             (N + c.bn - 1) / c.bn);
+    }
     int64_t m_blocks = (M + 127) / 128;
     int64_t pair_rows = (M + 255) / 256;
     if (layout == 2) {
@@ -966,6 +1214,7 @@ const char *dg_status_string(dg_status_t status)
     case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT";
     case DG_ERR_BAD_GROUP_DATA: return "DG_ERR_BAD_GROUP_DATA";
     case DG_ERR_WORKSPACE_LIMIT: return "DG_ERR_WORKSPACE_LIMIT";
+    case DG_ERR_BAD_SCALE: return "DG_ERR_BAD_SCALE";
     }
     return "DG_ERR_UNKNOWN";
 }

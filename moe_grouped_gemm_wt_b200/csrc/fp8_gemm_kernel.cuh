@@ -64,7 +64,9 @@ enum Layout : int { kDense = 0, kContiguous = 1, kMasked = 2, kKGrouped = 3 };
 // Device status word: code (bits 0-7), role (8-11), stage (12-19), CTA (20-31).
 constexpr uint32_t kCodeTimeout = 5;
 constexpr uint32_t kCodeBadGroup = 6;
-enum Role : uint32_t { kRoleProducer = 1, kRoleMma = 2, kRolePromote = 3, kRoleDrain = 4, kRoleSched = 5 };
+constexpr uint32_t kCodeBadScale = 8;
+enum Role : uint32_t { kRoleProducer = 1, kRoleMma = 2, kRolePromote = 3, kRoleDrain = 4, kRoleSched = 5,
+                       kRoleTransform = 6 };
 
 static __device__ unsigned int g_status_word = 0;
 
@@ -99,6 +101,11 @@ struct GemmParams {
     const float *C;
     float *D32;
     const int32_t *k_offsets;  // K-grouped only: [G+1] K-row offsets of the groups
+    // UE8M0 block-scaled mode: packed scales, four K blocks per int32.
+    const int32_t *sfa;  // dense/contig: [num_kg][sfa_ld]; masked: [G][num_kg][sfa_ld]
+    const int32_t *sfb;  // [G][num_kg][nbn]
+    int sfa_ld;          // padded row count of the packed LHS scales
+    int num_kg;          // ceil(num_kb / 4)
 };
 
 // Row segment of an fp32 output: drow[c] = acc[c] for the 4-float groups of

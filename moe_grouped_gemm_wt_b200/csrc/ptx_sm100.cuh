@@ -400,6 +400,32 @@ __device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc
         : "memory");
 }
 
+// Block-scaled MMA (kind::mxf8f6f4, one UE8M0 scale per row of A and per
+// row of B for each 32-wide K step): D[tmem] (+)= (A * sfa) * (B * sfb)^T.
+// sfa_tmem / sfb_tmem address the scale columns in TMEM (lane 0), with the
+// byte of each 32-bit scale word that this MMA uses in bits 30-31 (the same
+// byte index goes into the instruction descriptor).  Issued by one thread.
+__device__ __forceinline__ void mma_mxf8f6f4_bs(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Copies 32 rows x 16 bytes of shared memory (described by `sdesc`) into
+// TMEM lanes 0-31, four consecutive 32-bit columns from `taddr`, replicated
+// into each of the four 32-lane quarters (warpx4).  Asynchronous, ordered
+// with later tcgen05.mma of the same thread; tracked by tcgen05.commit.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Arrives once on the barrier at shared-memory offset `bar` in every CTA of
 // `cta_mask` when all pair MMAs previously issued by this thread have
 // completed (an arrive, not a data load: no multicast copy is involved).
@@ -482,6 +508,30 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t 
     d |= static_cast<uint64_t>(1) << 46;
     d |= static_cast<uint64_t>(2) << 61;
     return d;
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte scale chunk read by
+// tcgen05.cp: no swizzle, K-major, 8-row core matrices of 8 x 16 bytes laid
+// out back to back (stride-dimension offset 128 B; a single 16-byte column,
+// so the leading-dimension offset is never used and is left 0).  Version bit
+// 46 set, swizzle mode 0.
+__device__ __forceinline__ uint64_t smem_desc_sf_chunk(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+    d |= static_cast<uint64_t>(128 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    return d;
+}
+
+// Instruction descriptor for kind::mxf8f6f4 with block scaling: B's scale
+// byte in bits 4-5, A and B e4m3 (format 0 in bits 7-9 and 10-12), both
+// K-major, N >> 3 in bits 17-22, scale type UE8M0 (bit 23 = 1), M >> 4 in
+// bits 24-28, A's scale byte in bits 29-30; D is fp32.
+__host__ __device__ constexpr uint32_t idesc_mxf8_e4m3_ue8m0(int M, int N, uint32_t sf_byte)
+{
+    return ((sf_byte & 3u) << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(M >> 4) << 24) | ((sf_byte & 3u) << 29);
 }
 
 // Instruction descriptor for kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B

@@ -102,6 +102,48 @@ def test_null_and_alignment(lib):
     assert lib.dg_fp8_gemm_nt_acc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 512, None) == 0
 
 
+def test_ue8m0_validation(lib):
+    odd = ctypes.c_void_p(0x10008)
+    odd4 = ctypes.c_void_p(0x10004)
+    nt = lib.dg_fp8_gemm_nt_ue8m0
+    assert nt(None, FAKE, FAKE, FAKE, FAKE, 128, 256, 512, None) == 1
+    assert nt(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 250, 512, None) == 2
+    assert nt(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 500, None) == 2
+    assert nt(FAKE, odd4, FAKE, FAKE, FAKE, 128, 256, 512, None) == 3  # sfa: 16-byte aligned
+    assert nt(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 512, None) == 0
+    assert nt(FAKE, FAKE, FAKE, FAKE, FAKE, -1, 256, 512, None) == 1
+    cg = lib.dg_fp8_grouped_gemm_contiguous_ue8m0
+    assert cg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 200, 256, 512, 2, None) == 2
+    assert cg(FAKE, FAKE, FAKE, FAKE, FAKE, None, 256, 256, 512, 2, None) == 1
+    assert cg(FAKE, FAKE, odd, FAKE, FAKE, FAKE, 256, 256, 512, 2, None) == 3
+    assert cg(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 512, 2, None) == 0
+    mk = lib.dg_fp8_grouped_gemm_masked_ue8m0
+    assert mk(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 256, 512, 0, None) == 1
+    assert mk(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, -1, 256, 512, 0, None) == 1
+    assert mk(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 256, 256, 512, -1, None) == 1
+    assert mk(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0, 256, 512, 0, None) == 0
+    tr = lib.dg_transform_sf_ue8m0
+    assert tr(None, FAKE, 128, 512, 1, 1, None) == 1
+    assert tr(FAKE, FAKE, 128, 500, 1, 1, None) == 2
+    assert tr(FAKE, FAKE, 128, 512, 0, 1, None) == 1
+    assert tr(FAKE, FAKE, 128, 512, 1, 2, None) == 1
+    assert tr(FAKE, FAKE, 0, 512, 1, 0, None) == 0
+    assert lib.dg_status_string(8) == b"DG_ERR_BAD_SCALE"
+
+
+def test_ue8m0_describe_config(lib):
+    buf = ctypes.create_string_buffer(256)
+    for layout in (3, 4, 5):
+        assert lib.dg_describe_config(layout, 4096, 7168, 7168, 4, buf, 256) > 0
+        desc = dict(kv.split("=") for kv in buf.value.decode().split())
+        assert desc["ue8m0"] == "1" and desc["pair"] == "0" and desc["ksplit"] == "1"
+        assert int(desc["BN"]) in (128, 160, 192, 224)
+    # prefill shape: 32 m-blocks x 32 column tiles of 224 fill 148 SMs in 7 waves
+    lib.dg_describe_config(3, 4096, 7168, 18432, 1, buf, 256)
+    assert dict(kv.split("=") for kv in buf.value.decode().split())["BN"] == "224"
+    assert lib.dg_describe_config(6, 128, 256, 512, 1, buf, 256) == -1
+
+
 def test_sm_fill_example_from_pages(lib):
     """The unaligned-block-size example of the DeepGEMM article (lqnn.cn,
     section 非对齐块大小): M=256, N=7168 on 132 SMs -- 128x128 tiles occupy
