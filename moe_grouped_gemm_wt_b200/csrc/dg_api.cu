@@ -643,30 +643,94 @@ dg_status_t dense_gemm(const void *A, const float *sA, const void *B, const floa
 
 // ------------------------------------------------ UE8M0 block-scaled mode
 
-// Tile shapes of the block-scaled kernel.  The tensor core applies the
+// Tile shapes of the block-scaled kernels.  The tensor core applies the
 // scales, so a tile's time is its MMA time (proportional to BN) plus a fixed
-// fill/epilogue part; the planner takes the fewest waves x (BN + 48).
+// fill/epilogue part: cost = waves x (BN + 48) x feed, where feed > 1 for
+// one-CTA tiles, whose operand bytes per SM and K block ((128 + BN) x 128)
+// approach the L2 -> SM limit at full MMA rate; pair tiles (256 x BN on two
+// SMs, (128 + BN/2) x 128 bytes per SM) are taken when they fill every SM
+// pair.  dg_set_tile_family restricts the family as for the fp32-scale mode.
 struct BsChoice {
-    int bn, stages, ks;
+    int bn, stages, ks, pair;
+    double feed;
 };
-constexpr BsChoice kBsChoices[] = {{128, 3, 2}, {160, 2, 2}, {192, 2, 2}, {224, 2, 2}};
+constexpr BsChoice kBsChoices[] = {
+    {128, 3, 2, 0, 1.25}, {160, 2, 2, 0, 1.25}, {192, 2, 2, 0, 1.25}, {224, 2, 2, 0, 1.25},
+    {128, 4, 2, 1, 1.0},  {160, 3, 2, 1, 1.0},  {192, 3, 2, 1, 1.0},  {224, 3, 2, 1, 1.0},
+};
 
-BsChoice choose_bs(int64_t m_blocks, int N, int sms)
+BsChoice choose_bs(int64_t m_blocks, int64_t pair_rows, int N, int sms)
 {
     BsChoice best = kBsChoices[0];
     double best_cost = 1e300;
     for (const BsChoice &c : kBsChoices) {
         if (forced_block_n() > 0 && c.bn != forced_block_n())
             continue;
-        const int64_t tiles = m_blocks * ((N + c.bn - 1) / c.bn);
-        const int64_t waves = (tiles + sms - 1) / sms;
-        const double cost = static_cast<double>(waves) * (c.bn + 48);
+        if (forced_pair() >= 0 && c.pair != forced_pair())
+            continue;
+        const int units = c.pair ? sms / 2 : sms;
+        if (units <= 0)
+            continue;
+        const int64_t tiles = (c.pair ? pair_rows : m_blocks) * ((N + c.bn - 1) / c.bn);
+        if (c.pair && tiles < units && forced_pair() != 1)
+            continue;
+        const int64_t waves = (tiles + units - 1) / units;
+        const double cost = static_cast<double>(waves) * (c.bn + 48) * c.feed;
         if (cost < best_cost) {
             best_cost = cost;
             best = c;
         }
     }
     return best;
+}
+
+template <int BN, int STAGES, int KS, int LAYOUT>
+dg_status_t launch_bs_pair(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows, const GemmParams &p,
+                           int grid, cudaStream_t stream)
+{
+    using Cfg = dg::BsPairConfig<BN, STAGES, KS>;
+    CUtensorMap ta, tb, td64, tdrem;
+    if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
+        !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, Cfg::BN_HALF, KS))
+        return DG_ERR_CUDA;
+    if (!make_tmap_bf16(&td64, p.D, static_cast<uint64_t>(p.N), a_rows, 64, dg::kBM,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return DG_ERR_CUDA;
+    if (Cfg::EPI_REM > 0) {
+        if (!make_tmap_bf16(&tdrem, p.D, static_cast<uint64_t>(p.N), a_rows, Cfg::EPI_REM, dg::kBM,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+            return DG_ERR_CUDA;
+    } else {
+        tdrem = td64;
+    }
+    auto kern = dg::fp8_gemm_bs_pair_kernel<BN, STAGES, KS, LAYOUT>;
+    static std::atomic<bool> attr_set[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices)
+        return DG_ERR_CUDA;
+    if (!attr_set[dev].load()) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) !=
+            cudaSuccess)
+            return DG_ERR_CUDA;
+        attr_set[dev].store(true);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, td64, tdrem, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DG_ERR_CUDA;
+    }
+    return DG_OK;
 }
 
 template <int BN, int STAGES, int KS, int LAYOUT>
@@ -714,6 +778,28 @@ dg_status_t dispatch_bs(const BsChoice &c, const void *A, uint64_t a_rows, const
     p.num_nb = (p.N + c.bn - 1) / c.bn;
     p.ksplit = 1;
     p.kb_per_split = p.num_kb;
+    if (c.pair) {
+        // the pair scheduler counts 256-row pair rows
+        p.num_mb = (p.num_mb + 1) / 2;
+        if (LAYOUT != dg::kMasked)
+            p.raster = choose_raster(p.num_mb);
+        const int pairs = sms / 2;
+        const int64_t ptiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
+        int grid_pairs = pairs;
+        if (LAYOUT != dg::kMasked && ptiles < pairs)
+            grid_pairs = static_cast<int>(ptiles);
+        if (grid_pairs <= 0)
+            return DG_OK;
+#define DG_BS_PAIR_CASE(BN_, ST_, KS_)                                                              \
+        if (c.bn == BN_ && c.stages == ST_ && c.ks == KS_)                                           \
+            return launch_bs_pair<BN_, ST_, KS_, LAYOUT>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
+        DG_BS_PAIR_CASE(128, 4, 2)
+        DG_BS_PAIR_CASE(160, 3, 2)
+        DG_BS_PAIR_CASE(192, 3, 2)
+        DG_BS_PAIR_CASE(224, 3, 2)
+#undef DG_BS_PAIR_CASE
+        return DG_ERR_UNSUPPORTED;
+    }
     const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
     int grid = sms;
     if (LAYOUT != dg::kMasked)
@@ -1006,10 +1092,10 @@ dg_status_t dg_fp8_gemm_nt_ue8m0(const void *A, const int32_t *sfa, const void *
     if (sms <= 0)
         return DG_ERR_CUDA;
     GemmParams p = bs_params(sfa, sfb, D, M, N, K, 1);
-    const BsChoice c = choose_bs(p.num_mb, N, sms);
+    const BsChoice c = choose_bs(p.num_mb, (M + 255) / 256, N, sms);
     if (print_configs())
-        std::fprintf(stderr, "[dg] dense ue8m0 M=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n", M, N,
-                     K, c.bn, c.stages, c.ks, sms);
+        std::fprintf(stderr, "[dg] dense ue8m0 M=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d sms=%d\n", M, N,
+                     K, c.pair ? 256 : 128, c.bn, c.stages, c.ks, sms);
     return dispatch_bs<dg::kDense>(c, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), p, sms,
                                    stream);
 }
@@ -1037,10 +1123,10 @@ dg_status_t dg_fp8_grouped_gemm_contiguous_ue8m0(const void *A, const int32_t *s
         return DG_ERR_CUDA;
     GemmParams p = bs_params(sfa, sfb, D, M_total, N, K, num_groups);
     p.m_indices = m_indices;
-    const BsChoice c = choose_bs(p.num_mb, N, sms);
+    const BsChoice c = choose_bs(p.num_mb, (M_total + 255) / 256, N, sms);
     if (print_configs())
-        std::fprintf(stderr, "[dg] contiguous ue8m0 M=%d N=%d K=%d G=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
-                     M_total, N, K, num_groups, c.bn, c.stages, c.ks, sms);
+        std::fprintf(stderr, "[dg] contiguous ue8m0 M=%d N=%d K=%d G=%d -> BM=%d BN=%d stages=%d ks=%d sms=%d\n",
+                     M_total, N, K, num_groups, c.pair ? 256 : 128, c.bn, c.stages, c.ks, sms);
     return dispatch_bs<dg::kContiguous>(c, A, static_cast<uint64_t>(M_total), B,
                                         static_cast<uint64_t>(num_groups) * N, p, sms, stream);
 }
@@ -1069,11 +1155,12 @@ dg_status_t dg_fp8_grouped_gemm_masked_ue8m0(const void *A, const int32_t *sfa, 
     p.masked_m = masked_m;
     p.raster = 1;
     const int em = (expected_m > 0 && expected_m < max_m) ? expected_m : max_m;
-    const BsChoice c = choose_bs(static_cast<int64_t>(num_groups) * ((em + 127) / 128), N, sms);
+    const BsChoice c = choose_bs(static_cast<int64_t>(num_groups) * ((em + 127) / 128),
+                                 static_cast<int64_t>(num_groups) * ((em + 255) / 256), N, sms);
     if (print_configs())
         std::fprintf(stderr,
-                     "[dg] masked ue8m0 G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=128 BN=%d stages=%d ks=%d sms=%d\n",
-                     num_groups, max_m, em, N, K, c.bn, c.stages, c.ks, sms);
+                     "[dg] masked ue8m0 G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d sms=%d\n",
+                     num_groups, max_m, em, N, K, c.pair ? 256 : 128, c.bn, c.stages, c.ks, sms);
     return dispatch_bs<dg::kMasked>(c, A, static_cast<uint64_t>(num_groups) * max_m, B,
                                     static_cast<uint64_t>(num_groups) * N, p, sms, stream);
 }
@@ -1183,11 +1270,12 @@ int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, i
     if (layout >= 3) {
         // the UE8M0 block-scaled mode (one-CTA tiles, no K split)
         const int64_t mb = static_cast<int64_t>((M + 127) / 128) * (layout == 5 ? groups : 1);
-        const BsChoice c = choose_bs(mb, N, sms);
+        const int64_t pr = static_cast<int64_t>((M + 255) / 256) * (layout == 5 ? groups : 1);
+        const BsChoice c = choose_bs(mb, pr, N, sms);
         return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
-                             "layout=%d BM=128 BN=%d BK=128 stages=%d ks=%d ksplit=1 pair=0 wg=1 sms=%d m_blocks=%lld n_blocks=%d ue8m0=1",
-                             layout, c.bn, c.stages, c.ks, sms, static_cast<long long>(mb),
-                             (N + c.bn - 1) / c.bn);
+                             "layout=%d BM=%d BN=%d BK=128 stages=%d ks=%d ksplit=1 pair=%d wg=1 sms=%d m_blocks=%lld n_blocks=%d ue8m0=1",
+                             layout, c.pair ? 256 : 128, c.bn, c.stages, c.ks, c.pair, sms,
+                             static_cast<long long>(c.pair ? pr : mb), (N + c.bn - 1) / c.bn);
     }
     int64_t m_blocks = (M + 127) / 128;
     int64_t pair_rows = (M + 255) / 256;

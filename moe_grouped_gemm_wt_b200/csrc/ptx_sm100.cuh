@@ -131,6 +131,29 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster)
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
+// Remote arrive with release semantics at cluster scope: this thread's
+// earlier writes (to its own CTA's shared memory) are visible to a thread of
+// the cluster that acquires the phase at cluster scope.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t bar_cluster)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// As mbar_try_wait, acquiring at cluster scope (pairs with
+// mbar_arrive_release_cluster from the peer CTA).
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // True once the phase with parity `parity` has completed.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
@@ -238,6 +261,38 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v)
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// 4-byte asynchronous global->shared copy; src_bytes = 0 zero-fills the
+// destination without reading global memory.
+__device__ __forceinline__ void cp_async_4_zfill(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+// Closes this thread's current group of cp.async copies.
+__device__ __forceinline__ void cp_async_commit_group()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Waits until at most N of this thread's most recent cp.async groups are
+// still pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4u(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
 }
 
 // 16-byte asynchronous global->shared copy; src_bytes = 0 zero-fills the
@@ -415,6 +470,31 @@ __device__ __forceinline__ void mma_mxf8f6f4_bs(uint32_t d_tmem, uint64_t a_desc
         "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
         : "memory");
+}
+
+// Pair form of mma_mxf8f6f4_bs (cta_group::2, M = 256), issued by one thread
+// of the pair's rank-0 CTA: A's rows 0-127 and the first N/2 rows of B come
+// from rank 0's shared memory, the rest from rank 1's; each CTA's TMEM holds
+// the scales of its own 128 rows of A and of all N rows of B, at the same
+// TMEM addresses, and receives its 128 rows of D.
+__device__ __forceinline__ void mma_mxf8f6f4_bs_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                     uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                     uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Pair form of tmem_cp_32x128b_warpx4 (cta_group::2), issued by rank 0: each
+// CTA of the pair copies from its own shared memory at the descriptor's
+// address into its own TMEM at `taddr`.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Copies 32 rows x 16 bytes of shared memory (described by `sdesc`) into

@@ -136,11 +136,16 @@ def test_ue8m0_describe_config(lib):
     for layout in (3, 4, 5):
         assert lib.dg_describe_config(layout, 4096, 7168, 7168, 4, buf, 256) > 0
         desc = dict(kv.split("=") for kv in buf.value.decode().split())
-        assert desc["ue8m0"] == "1" and desc["pair"] == "0" and desc["ksplit"] == "1"
+        assert desc["ue8m0"] == "1" and desc["ksplit"] == "1"
         assert int(desc["BN"]) in (128, 160, 192, 224)
-    # prefill shape: 32 m-blocks x 32 column tiles of 224 fill 148 SMs in 7 waves
+    # prefill shape: 16 pair rows x 32 column tiles of 224 fill 74 SM pairs
+    # in 7 waves (98.8% of the last wave used)
     lib.dg_describe_config(3, 4096, 7168, 18432, 1, buf, 256)
-    assert dict(kv.split("=") for kv in buf.value.decode().split())["BN"] == "224"
+    desc = dict(kv.split("=") for kv in buf.value.decode().split())
+    assert (desc["BN"], desc["BM"], desc["pair"]) == ("224", "256", "1")
+    # decode shape: too few pair tiles to fill the pairs, one-CTA tiles
+    lib.dg_describe_config(3, 128, 2112, 7168, 1, buf, 256)
+    assert dict(kv.split("=") for kv in buf.value.decode().split())["pair"] == "0"
     assert lib.dg_describe_config(6, 128, 256, 512, 1, buf, 256) == -1
 
 

@@ -5,10 +5,12 @@ summary, section "Giao dien GEMM va rang buoc layout").
 Inputs are quantised with power-of-two scales (the input recipe's ue8m0
 option, whose rounding the CPU suite checks against the oracle), packed on
 the GPU by dg_transform_sf_ue8m0 (checked word for word against the oracle's
-packing) and multiplied by the block-scaled kernel.  Shapes are chosen, with
-the SM count capped at 16 for the small ones, so that every compiled tile
-width runs, with ragged M and N, partial K-block groups (K/128 not a
-multiple of 4), several waves of tiles, grouped padding and masking.
+packing) and multiplied by the block-scaled kernels, on one-CTA tiles and on
+CTA-pair tiles (cta_group::2).  Shapes are chosen, with the SM count capped
+at 16 for the small ones, so that every compiled tile width runs, with
+ragged M and N, partial K-block groups (K/128 not a multiple of 4), several
+waves of tiles, pairs whose halves belong to different groups, grouped
+padding and masking.
 Placement and masking are bit-exact (sentinel pre-fill)."""
 import numpy as np
 import pytest
@@ -70,6 +72,15 @@ def _dense(dg, oracle_mod, p):
     return bits(D), (A, sfa, B, sfb, D)
 
 
+@pytest.fixture(params=[1, 2], ids=["one_cta", "pair"])
+def family(request, dg):
+    """Runs a test on one tile family (dg_set_tile_family: 1 = one-CTA
+    128-row tiles, 2 = CTA-pair 256-row tiles)."""
+    dg.dg_set_tile_family(request.param)
+    yield request.param
+    dg.dg_set_tile_family(dg.DG_TILES_AUTO)
+
+
 @pytest.mark.parametrize("M,N,K,bn", [
     (2048, 224, 512, "224"),   # 16 tiles of 224 on 16 SMs
     (2048, 192, 896, "192"),   # 7 K blocks: the last word holds 3
@@ -79,10 +90,11 @@ def _dense(dg, oracle_mod, p):
     (130, 2064, 640, None),    # second m-block has 2 rows
     (384, 7168, 1152, None),   # wide N, 9 K blocks
 ])
-def test_dense_ue8m0_matches_oracle(dg, oracle_mod, M, N, K, bn):
+def test_dense_ue8m0_matches_oracle(dg, oracle_mod, family, M, N, K, bn):
     dg.dg_set_num_sms(CAP_SMS)
     try:
         plan = _plan(dg, 3, M, N, K)
+        assert plan["pair"] == ("1" if family == 2 else "0"), plan
         if bn is not None:
             assert plan["BN"] == bn, plan
         p = gi.dense_problem(M, N, K, seed_a=5000 + M, seed_b=6000 + N, ue8m0=True)
@@ -94,7 +106,7 @@ def test_dense_ue8m0_matches_oracle(dg, oracle_mod, M, N, K, bn):
     assert_close(got, ref, f"ue8m0 dense {M}x{N}x{K}")
 
 
-def test_dense_ue8m0_integer_inputs_bit_exact(dg, oracle_mod):
+def test_dense_ue8m0_integer_inputs_bit_exact(dg, oracle_mod, family):
     """Integer-valued codes with power-of-two scales: every partial and every
     scaled sum is exact in fp32, so the bf16 result equals the oracle's bit
     for bit."""
@@ -124,7 +136,7 @@ def test_ue8m0_and_fp32_modes_agree(dg, oracle_mod):
     assert_close(got_bs, bits(D), "ue8m0 vs fp32-scale mode")
 
 
-def test_dense_ue8m0_deterministic(dg, oracle_mod):
+def test_dense_ue8m0_deterministic(dg, oracle_mod, family):
     p = gi.dense_problem(384, 2112, 1024, seed_a=73, seed_b=74, ue8m0=True)
     a, _ = _dense(dg, oracle_mod, p)
     b, _ = _dense(dg, oracle_mod, p)
@@ -156,9 +168,10 @@ def test_dense_prefill_ue8m0_sampled(dg, oracle_mod):
 @pytest.mark.parametrize("rows,N,K", [
     ([384, 100, 300], 1024, 512),     # padded blocks, ragged groups
     ([0, 640, 37], 1040, 256),        # an empty group, ragged N
-    ([128] * 6, 224, 1152),           # many groups, 9 K blocks
+    ([128] * 6, 224, 1152),           # many groups, 9 K blocks; every pair spans two groups
+    ([256, 128, 384], 448, 640),      # pairs split across groups and padding
 ])
-def test_contiguous_ue8m0_matches_oracle(dg, oracle_mod, rows, N, K):
+def test_contiguous_ue8m0_matches_oracle(dg, oracle_mod, family, rows, N, K):
     p = gi.contiguous_problem(rows, N, K, seed_a=81, seed_b=82, ue8m0=True)
     dev = torch.device("cuda")
     A = torch.from_numpy(p["A"]).to(dev)
@@ -182,7 +195,7 @@ def test_contiguous_ue8m0_matches_oracle(dg, oracle_mod, rows, N, K):
     (3, 200, 2064, 640, [200, 129, 1]),   # max_m not a multiple of 128
     (2, 256, 224, 128, [256, 255]),
 ])
-def test_masked_ue8m0_matches_oracle(dg, oracle_mod, G, max_m, N, K, masked):
+def test_masked_ue8m0_matches_oracle(dg, oracle_mod, family, G, max_m, N, K, masked):
     p = gi.masked_problem(G, max_m, N, K, masked_m=masked, seed_a=91, seed_b=92, ue8m0=True)
     dev = torch.device("cuda")
     A = torch.from_numpy(p["A"]).to(dev)
