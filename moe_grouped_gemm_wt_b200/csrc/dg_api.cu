@@ -684,14 +684,14 @@ BsChoice choose_bs(int64_t m_blocks, int64_t pair_rows, int N, int sms)
     return best;
 }
 
-template <int BN, int STAGES, int KS, int LAYOUT>
-dg_status_t launch_bs_pair(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows, const GemmParams &p,
-                           int grid, cudaStream_t stream)
+template <int BN, int STAGES, int KS, int LAYOUT, bool PAIR>
+dg_status_t launch_bs(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows, const GemmParams &p,
+                      int grid, cudaStream_t stream)
 {
-    using Cfg = dg::BsPairConfig<BN, STAGES, KS>;
+    using Cfg = dg::BsConfig<BN, STAGES, KS, PAIR>;
     CUtensorMap ta, tb, td64, tdrem;
     if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
-        !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, Cfg::BN_HALF, KS))
+        !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, Cfg::B_ROWS, KS))
         return DG_ERR_CUDA;
     if (!make_tmap_bf16(&td64, p.D, static_cast<uint64_t>(p.N), a_rows, 64, dg::kBM,
                         CU_TENSOR_MAP_SWIZZLE_128B))
@@ -703,7 +703,7 @@ dg_status_t launch_bs_pair(const void *A, uint64_t a_rows, const void *B, uint64
     } else {
         tdrem = td64;
     }
-    auto kern = dg::fp8_gemm_bs_pair_kernel<BN, STAGES, KS, LAYOUT>;
+    auto kern = dg::fp8_gemm_bs_kernel<BN, STAGES, KS, LAYOUT, PAIR>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices)
@@ -721,50 +721,12 @@ dg_status_t launch_bs_pair(const void *A, uint64_t a_rows, const void *B, uint64
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.x = PAIR ? 2 : 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = PAIR ? 1 : 0;
     if (cudaLaunchKernelEx(&cfg, kern, ta, tb, td64, tdrem, p) != cudaSuccess) {
-        (void)cudaGetLastError();
-        return DG_ERR_CUDA;
-    }
-    return DG_OK;
-}
-
-template <int BN, int STAGES, int KS, int LAYOUT>
-dg_status_t launch_bs(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows, const GemmParams &p,
-                      int grid, cudaStream_t stream)
-{
-    using Cfg = dg::BsConfig<BN, STAGES, KS>;
-    CUtensorMap ta, tb, td64, tdrem;
-    if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
-        !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, BN, KS))
-        return DG_ERR_CUDA;
-    if (!make_tmap_bf16(&td64, p.D, static_cast<uint64_t>(p.N), a_rows, 64, dg::kBM,
-                        CU_TENSOR_MAP_SWIZZLE_128B))
-        return DG_ERR_CUDA;
-    if (Cfg::EPI_REM > 0) {
-        if (!make_tmap_bf16(&tdrem, p.D, static_cast<uint64_t>(p.N), a_rows, Cfg::EPI_REM, dg::kBM,
-                            CU_TENSOR_MAP_SWIZZLE_NONE))
-            return DG_ERR_CUDA;
-    } else {
-        tdrem = td64;
-    }
-    auto kern = dg::fp8_gemm_bs_kernel<BN, STAGES, KS, LAYOUT>;
-    static std::atomic<bool> attr_set[kMaxDevices];
-    const int dev = current_device();
-    if (dev < 0 || dev >= kMaxDevices)
-        return DG_ERR_CUDA;
-    if (!attr_set[dev].load()) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) !=
-            cudaSuccess)
-            return DG_ERR_CUDA;
-        attr_set[dev].store(true);
-    }
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, td64, tdrem, p);
-    if (cudaPeekAtLastError() != cudaSuccess) {
         (void)cudaGetLastError();
         return DG_ERR_CUDA;
     }
@@ -792,7 +754,7 @@ dg_status_t dispatch_bs(const BsChoice &c, const void *A, uint64_t a_rows, const
             return DG_OK;
 #define DG_BS_PAIR_CASE(BN_, ST_, KS_)                                                              \
         if (c.bn == BN_ && c.stages == ST_ && c.ks == KS_)                                           \
-            return launch_bs_pair<BN_, ST_, KS_, LAYOUT>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
+            return launch_bs<BN_, ST_, KS_, LAYOUT, true>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
         DG_BS_PAIR_CASE(128, 4, 2)
         DG_BS_PAIR_CASE(160, 3, 2)
         DG_BS_PAIR_CASE(192, 3, 2)
@@ -808,7 +770,7 @@ dg_status_t dispatch_bs(const BsChoice &c, const void *A, uint64_t a_rows, const
         return DG_OK;
 #define DG_BS_CASE(BN_, ST_, KS_)                                                                   \
     if (c.bn == BN_ && c.stages == ST_ && c.ks == KS_)                                               \
-        return launch_bs<BN_, ST_, KS_, LAYOUT>(A, a_rows, B, b_rows, p, grid, stream);
+        return launch_bs<BN_, ST_, KS_, LAYOUT, false>(A, a_rows, B, b_rows, p, grid, stream);
     DG_BS_CASE(128, 3, 2)
     DG_BS_CASE(160, 2, 2)
     DG_BS_CASE(192, 2, 2)

@@ -131,29 +131,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster)
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
-// Remote arrive with release semantics at cluster scope: this thread's
-// earlier writes (to its own CTA's shared memory) are visible to a thread of
-// the cluster that acquires the phase at cluster scope.
-__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t bar_cluster)
-{
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
-}
-
-// As mbar_try_wait, acquiring at cluster scope (pairs with
-// mbar_arrive_release_cluster from the peer CTA).
-__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // True once the phase with parity `parity` has completed.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
@@ -489,23 +466,6 @@ __device__ __forceinline__ void mma_mxf8f6f4_bs_pair(uint32_t d_tmem, uint64_t a
         : "memory");
 }
 
-// Pair form of tmem_cp_32x128b_warpx4 (cta_group::2), issued by rank 0: each
-// CTA of the pair copies from its own shared memory at the descriptor's
-// address into its own TMEM at `taddr`.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4_pair(uint32_t taddr, uint64_t sdesc)
-{
-    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-// Copies 32 rows x 16 bytes of shared memory (described by `sdesc`) into
-// TMEM lanes 0-31, four consecutive 32-bit columns from `taddr`, replicated
-// into each of the four 32-lane quarters (warpx4).  Asynchronous, ordered
-// with later tcgen05.mma of the same thread; tracked by tcgen05.commit.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc)
-{
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 // Arrives once on the barrier at shared-memory offset `bar` in every CTA of
 // `cta_mask` when all pair MMAs previously issued by this thread have
 // completed (an arrive, not a data load: no multicast copy is involved).
@@ -550,6 +510,21 @@ __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[
         : "r"(taddr));
 }
 
+// 32 lanes x 4 consecutive 32-bit columns: thread i of the warp writes v to
+// lane (taddr.lane + i), columns taddr.col .. taddr.col+3.  Whole warp.
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Waits until this thread's tcgen05.st have completed.
+__device__ __forceinline__ void tmem_st_wait()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait()
 {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -587,20 +562,6 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t 
     d |= static_cast<uint64_t>(1024 >> 4) << 32;
     d |= static_cast<uint64_t>(1) << 46;
     d |= static_cast<uint64_t>(2) << 61;
-    return d;
-}
-
-// Shared-memory descriptor of a 32-row x 16-byte scale chunk read by
-// tcgen05.cp: no swizzle, K-major, 8-row core matrices of 8 x 16 bytes laid
-// out back to back (stride-dimension offset 128 B; a single 16-byte column,
-// so the leading-dimension offset is never used and is left 0).  Version bit
-// 46 set, swizzle mode 0.
-__device__ __forceinline__ uint64_t smem_desc_sf_chunk(uint32_t saddr)
-{
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
-    d |= static_cast<uint64_t>(128 >> 4) << 32;
-    d |= static_cast<uint64_t>(1) << 46;
     return d;
 }
 
