@@ -18,6 +18,12 @@ the max over ranks and the value counts the work of all ranks.
 
 --impl reference times the CPU oracle (the only reference that exists for
 this method) on the same workload and metric, rank 0 only.
+
+--scales ue8m0 times the separately declared UE8M0 block-scaled mode instead
+(inputs quantised with power-of-two scales, packed four to an int32; the
+tensor core applies them).  The default run also reports that mode's
+per-shape numbers under "ue8m0_shapes"; the headline stays the fp32-scale
+mode.
 """
 from __future__ import annotations
 
@@ -100,14 +106,14 @@ def kernel_hash():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload):
+def ncu_traffic(workload, ue8m0=False):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
     on the current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
-        e = t.get(workload)
+        e = t.get(workload + (":ue8m0" if ue8m0 else ""))
         if e and e.get("kernel_hash") == kernel_hash():
             return float(e["dram_bytes_per_launch"])
     except (OSError, ValueError):
@@ -180,7 +186,15 @@ class ClockSampler:
 
 # ------------------------------------------------------------ our library
 
-def to_device(p, torch, dev):
+def pack_ue8m0(dg, p, d):
+    """The UE8M0 mode's packed scale words, built on the device from the
+    fp32 power-of-two scales (dg_transform_sf_ue8m0)."""
+    rows = p["M"] if p["kind"] != "masked" else p["max_m"]
+    d["sfa"] = dg.dg_transform_sf_ue8m0(d["sA"], rows, mn_major=True)
+    d["sfb"] = dg.dg_transform_sf_ue8m0(d["sB"], d["sB"].shape[-2], mn_major=False)
+
+
+def to_device(p, torch, dev, dg=None):
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
     out = dict(A=t(p["A"]), B=t(p["B"]), sA=t(gi.sa_to_kernel_layout(p["sA"])), sB=t(p["sB"]))
     if p["kind"] == "dense":
@@ -191,10 +205,22 @@ def to_device(p, torch, dev):
     else:
         out["masked_m"] = t(p["masked_m"])
         out["D"] = torch.empty((p["G"], p["max_m"], p["N"]), dtype=torch.bfloat16, device=dev)
+    if p.get("ue8m0"):
+        pack_ue8m0(dg, p, out)
     return out
 
 
 def call(dg, p, d, stream=None):
+    if p.get("ue8m0"):
+        if p["kind"] == "dense":
+            dg.dg_fp8_gemm_nt_ue8m0(d["A"], d["sfa"], d["B"], d["sfb"], d["D"], stream=stream)
+        elif p["kind"] == "contiguous":
+            dg.dg_fp8_grouped_gemm_contiguous_ue8m0(d["A"], d["sfa"], d["B"], d["sfb"], d["D"],
+                                                    d["m_indices"], stream=stream)
+        else:
+            dg.dg_fp8_grouped_gemm_masked_ue8m0(d["A"], d["sfa"], d["B"], d["sfb"], d["D"], d["masked_m"],
+                                                expected_m=int(np.mean(p["masked_m"])), stream=stream)
+        return
     if p["kind"] == "dense":
         dg.dg_fp8_gemm_nt(d["A"], d["sA"], d["B"], d["sB"], d["D"], stream=stream)
     elif p["kind"] == "contiguous":
@@ -257,11 +283,18 @@ def workload_label(p, name):
 
 
 def tile_label(dg, p):
+    base = 3 if p.get("ue8m0") else 0  # describe_config layouts 3-5: the UE8M0 mode
     if p["kind"] == "dense":
-        return dg.dg_describe_config(0, p["M"], p["N"], p["K"], 1)
+        return dg.dg_describe_config(base, p["M"], p["N"], p["K"], 1)
     if p["kind"] == "contiguous":
-        return dg.dg_describe_config(1, p["M"], p["N"], p["K"], p["G"])
-    return dg.dg_describe_config(2, int(np.mean(p["masked_m"])), p["N"], p["K"], p["G"])
+        return dg.dg_describe_config(base + 1, p["M"], p["N"], p["K"], p["G"])
+    return dg.dg_describe_config(base + 2, int(np.mean(p["masked_m"])), p["N"], p["K"], p["G"])
+
+
+def make_problem(name, ue8m0):
+    p = gi.make_workload(name, ue8m0=ue8m0)
+    p["ue8m0"] = ue8m0
+    return p
 
 
 def time_kernel(torch, dg, p, d, steps, warmup, flush):
@@ -291,7 +324,7 @@ def time_e2e(torch, dg, p, steps, warmup, dev):
     host = {k: torch.from_numpy(np.ascontiguousarray(v)).pin_memory()
             for k, v in (("A", p["A"]), ("B", p["B"]), ("sA", gi.sa_to_kernel_layout(p["sA"])),
                          ("sB", p["sB"]))}
-    d = to_device(p, torch, dev)
+    d = to_device(p, torch, dev, dg)
     out_host = torch.empty(d["D"].shape, dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host.numel() * out_host.element_size()
@@ -300,6 +333,8 @@ def time_e2e(torch, dg, p, steps, warmup, dev):
     def one():
         for k in host:
             d[k].copy_(host[k], non_blocking=True)
+        if p.get("ue8m0"):
+            pack_ue8m0(dg, p, d)  # the scale packing is part of the user's call path
         call(dg, p, d)
         out_host.copy_(d["D"], non_blocking=True)
 
@@ -391,7 +426,8 @@ def run_ours(args):
     pk = peaks()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
-    p = gi.make_workload(args.workload)
+    ue8m0 = args.scales == "ue8m0"
+    p = make_problem(args.workload, ue8m0)
     # Grouped workloads on several ranks: expert parallel, the fixed problem
     # split by expert (strong scaling); dense workloads: one replica per rank
     # (weak scaling).
@@ -401,7 +437,7 @@ def run_ours(args):
         if world > p["G"]:
             raise SystemExit(f"expert parallel: {world} ranks for {p['G']} experts")
         p = shard_experts(p, rank, world)
-    d = to_device(p, torch, dev)
+    d = to_device(p, torch, dev, dg)
     flop, byts, _ = workload_cost(p)
 
     sampler = ClockSampler(local)
@@ -415,26 +451,35 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
 
-    # per-shape sweep (every rank runs it; rank 0 reports)
-    shapes = {}
-    if not args.no_shapes:
+    # per-shape sweeps (every rank runs them; rank 0 reports): the mode
+    # timed above, and, after a default fp32-scale run, the UE8M0 mode too
+    def sweep(sweep_ue8m0):
+        out = {}
         for name in gi.WORKLOADS:
-            same = name == args.workload and not expert_parallel  # a shard is not the shape
-            q = p if same else gi.make_workload(name)
-            dq = d if same else to_device(q, torch, dev)
+            # a shard is not the shape
+            same = name == args.workload and not expert_parallel and sweep_ue8m0 == ue8m0
+            q = p if same else make_problem(name, sweep_ue8m0)
+            dq = d if same else to_device(q, torch, dev, dg)
             tq = time_kernel(torch, dg, q, dq, max(10, min(args.steps, 30)), 3, flush)
             mq = statistics.median(tq)
             fq, bq, rows = workload_cost(q)
             bound, t_roof, _ = roofline(fq, bq, pk)
-            shapes[name] = {
+            out[name] = {
                 "us": mq * 1e3, "tflops": fq / (mq * 1e-3) / 1e12,
                 "bound": bound, "roofline_us": t_roof * 1e6,
                 "frac_of_roofline": t_roof / (mq * 1e-3),
-                "valid_rows": rows,
+                "valid_rows": rows, "tile": tile_label(dg, q),
             }
             if not same:
                 del dq
                 torch.cuda.empty_cache()
+        return out
+
+    shapes, ue8m0_shapes = {}, None
+    if not args.no_shapes:
+        shapes = sweep(ue8m0)
+        if not ue8m0 and not args.no_ue8m0_shapes:
+            ue8m0_shapes = sweep(True)
     clocks = sampler.stop()
 
     e2e_ms, h2d, d2h = time_e2e(torch, dg, p, max(10, min(args.steps, 50)), 3, dev)
@@ -449,7 +494,7 @@ def run_ours(args):
         achieved = flop / (ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp8_peak}
-    roof["traffic"] = ncu_traffic(args.workload)
+    roof["traffic"] = ncu_traffic(args.workload, ue8m0)
     roof["peak_source"] = pk["source"] + (" (fp8 = 2 x measured bf16)" if bound == "tensor" else "")
 
     cpu = None
@@ -467,13 +512,18 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
         "higher_is_better": True, "scaling": "strong" if expert_parallel else "weak",
-        "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 promotion, bf16 out)",
-        "data": "synthetic (seeded N(0,1) quantised to e4m3 with 1x128 / 128x128 fp32 scales)",
+        "vs_baseline": None,
+        "dtype": ("fp8_e4m3 (UE8M0 block-scaled MMA, fp32 accumulate, bf16 out)" if ue8m0
+                  else "fp8_e4m3 (fp32 promotion, bf16 out)"),
+        "data": ("synthetic (seeded N(0,1) quantised to e4m3 with 1x128 / 128x128 power-of-two scales, "
+                 "packed UE8M0)" if ue8m0 else
+                 "synthetic (seeded N(0,1) quantised to e4m3 with 1x128 / 128x128 fp32 scales)"),
         "config": {"workload": workload_label(p, args.workload),
                    "l2": "flushed before every timed launch (512 MiB write)",
                    "parallelism": (f"expert parallel x{world} (this rank: {p['G']} experts)"
                                    if expert_parallel else f"replicas x{world}"),
-                   "tile": tile_label(dg, p)},
+                   "tile": tile_label(dg, p),
+                   "scales": "ue8m0 (separately declared block-scaled mode)" if ue8m0 else "fp32"},
         "roofline": roof,
         "frac_of_roofline": t_roof / (ms * 1e-3),
         "cpu_baseline": cpu,
@@ -483,6 +533,8 @@ def run_ours(args):
         "clocks": clocks,
         "shapes": shapes,
     }
+    if ue8m0_shapes is not None:
+        line["ue8m0_shapes"] = ue8m0_shapes
     print(json.dumps(line), flush=True)
     return 0
 
@@ -496,6 +548,10 @@ def main():
     ap.add_argument("--no-shapes", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--scales", choices=("fp32", "ue8m0"), default="fp32",
+                    help="fp32 scales (the headline mode) or the UE8M0 block-scaled mode")
+    ap.add_argument("--no-ue8m0-shapes", action="store_true",
+                    help="skip the UE8M0 mode's per-shape sweep of a default run")
     ap.add_argument("--workload", choices=sorted(gi.WORKLOADS), default=HEADLINE,
                     help="workload timed as the step (default: the decode-shaped dense GEMM)")
     args = ap.parse_args()

@@ -314,9 +314,18 @@ Plan choose_plan(int64_t m_blocks, int64_t pair_rows, int N, int num_kb, int sms
     return best;
 }
 
+// Rasterisation: tiles are visited in groups of `raster` m-block rows (pair
+// rows for pair tiles), column by column inside a group.  DG_RASTER=<n>
+// overrides the group height (read once; for tuning sweeps).
 int choose_raster(int num_mb)
 {
-    return num_mb < 16 ? (num_mb > 0 ? num_mb : 1) : 16;
+    static int forced = -1;
+    if (forced < 0) {
+        const char *e = std::getenv("DG_RASTER");
+        forced = e ? std::atoi(e) : 0;
+    }
+    const int want = forced > 0 ? forced : 16;
+    return num_mb < want ? (num_mb > 0 ? num_mb : 1) : want;
 }
 
 template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false>
@@ -682,6 +691,17 @@ BsChoice choose_bs(int64_t m_blocks, int64_t pair_rows, int N, int sms)
         }
     }
     return best;
+}
+
+// Masked (decode) problems are HBM-bound: the one-CTA 128-column tile, whose
+// three-stage ring keeps the most bytes in flight, measured best (129 us on
+// 16 x 256 x 4096 x 7168 against 140-162 us for the other shapes); an
+// explicit tile-family or width restriction still goes through choose_bs.
+BsChoice choose_bs_masked(int64_t m_blocks, int64_t pair_rows, int N, int sms)
+{
+    if (forced_block_n() <= 0 && forced_pair() < 0)
+        return kBsChoices[0];
+    return choose_bs(m_blocks, pair_rows, N, sms);
 }
 
 template <int BN, int STAGES, int KS, int LAYOUT, bool PAIR>
@@ -1117,8 +1137,8 @@ dg_status_t dg_fp8_grouped_gemm_masked_ue8m0(const void *A, const int32_t *sfa, 
     p.masked_m = masked_m;
     p.raster = 1;
     const int em = (expected_m > 0 && expected_m < max_m) ? expected_m : max_m;
-    const BsChoice c = choose_bs(static_cast<int64_t>(num_groups) * ((em + 127) / 128),
-                                 static_cast<int64_t>(num_groups) * ((em + 255) / 256), N, sms);
+    const BsChoice c = choose_bs_masked(static_cast<int64_t>(num_groups) * ((em + 127) / 128),
+                                        static_cast<int64_t>(num_groups) * ((em + 255) / 256), N, sms);
     if (print_configs())
         std::fprintf(stderr,
                      "[dg] masked ue8m0 G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d sms=%d\n",
@@ -1230,10 +1250,10 @@ int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, i
     if (sms <= 0)
         sms = g_num_sms_cap.load() > 0 ? g_num_sms_cap.load() : 148;
     if (layout >= 3) {
-        // the UE8M0 block-scaled mode (one-CTA tiles, no K split)
+        // the UE8M0 block-scaled mode (one-CTA or pair tiles, no K split)
         const int64_t mb = static_cast<int64_t>((M + 127) / 128) * (layout == 5 ? groups : 1);
         const int64_t pr = static_cast<int64_t>((M + 255) / 256) * (layout == 5 ? groups : 1);
-        const BsChoice c = choose_bs(mb, pr, N, sms);
+        const BsChoice c = layout == 5 ? choose_bs_masked(mb, pr, N, sms) : choose_bs(mb, pr, N, sms);
         return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
                              "layout=%d BM=%d BN=%d BK=128 stages=%d ks=%d ksplit=1 pair=%d wg=1 sms=%d m_blocks=%lld n_blocks=%d ue8m0=1",
                              layout, c.pair ? 256 : 128, c.bn, c.stages, c.ks, c.pair, sms,
