@@ -662,7 +662,15 @@ dg_status_t dense_gemm(const void *A, const float *sA, const void *B, const floa
 struct BsChoice {
     int bn, stages, ks, pair;
     double feed;
+    int ksplit = 1;  // > 1: the dense K-split kernel, a cluster of ksplit CTAs per tile
 };
+
+// The dense decode plan of the UE8M0 mode: problems with too few tiles to
+// fill the GPU split each 128 x 144 tile's K range over a cluster of S CTAs
+// (S = 8, 4 or 2: the largest that leaves every split two K blocks and keeps
+// all of the grid's clusters co-resident).
+constexpr int kBsSplitBN = 144;
+int bs_split_max_clusters(int S);
 constexpr BsChoice kBsChoices[] = {
     {128, 3, 2, 0, 1.25}, {160, 2, 2, 0, 1.25}, {192, 2, 2, 0, 1.25}, {224, 2, 2, 0, 1.25},
     {128, 4, 2, 1, 1.0},  {160, 3, 2, 1, 1.0},  {192, 3, 2, 1, 1.0},  {224, 3, 2, 1, 1.0},
@@ -693,6 +701,27 @@ BsChoice choose_bs(int64_t m_blocks, int64_t pair_rows, int N, int sms)
     return best;
 }
 
+BsChoice choose_bs_dense(int64_t m_blocks, int64_t pair_rows, int N, int num_kb, int sms)
+{
+    BsChoice c = choose_bs(m_blocks, pair_rows, N, sms);
+    if (forced_block_n() > 0 || forced_pair() == 1)
+        return c;
+    const int64_t tiles = m_blocks * ((N + c.bn - 1) / c.bn);
+    if (c.pair || tiles * 2 > sms)
+        return c;
+    const int64_t split_tiles = m_blocks * ((N + kBsSplitBN - 1) / kBsSplitBN);
+    for (int S = 8; S >= 2; S /= 2) {
+        const int kbps = (num_kb + S - 1) / S;
+        if (kbps < 2 || (num_kb + kbps - 1) / kbps != S)
+            continue;
+        if (split_tiles > bs_split_max_clusters(S))
+            continue;
+        BsChoice sc{kBsSplitBN, 3, 2, 0, 1.0, S};
+        return sc;
+    }
+    return c;
+}
+
 // Masked (decode) problems are HBM-bound: the one-CTA 128-column tile, whose
 // three-stage ring keeps the most bytes in flight, measured best (129 us on
 // 16 x 256 x 4096 x 7168 against 140-162 us for the other shapes); an
@@ -704,11 +733,11 @@ BsChoice choose_bs_masked(int64_t m_blocks, int64_t pair_rows, int N, int sms)
     return choose_bs(m_blocks, pair_rows, N, sms);
 }
 
-template <int BN, int STAGES, int KS, int LAYOUT, bool PAIR>
+template <int BN, int STAGES, int KS, int LAYOUT, bool PAIR, bool SPLIT = false>
 dg_status_t launch_bs(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows, const GemmParams &p,
                       int grid, cudaStream_t stream)
 {
-    using Cfg = dg::BsConfig<BN, STAGES, KS, PAIR>;
+    using Cfg = dg::BsConfig<BN, STAGES, KS, PAIR, SPLIT>;
     CUtensorMap ta, tb, td64, tdrem;
     if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
         !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, Cfg::B_ROWS, KS))
@@ -723,7 +752,7 @@ dg_status_t launch_bs(const void *A, uint64_t a_rows, const void *B, uint64_t b_
     } else {
         tdrem = td64;
     }
-    auto kern = dg::fp8_gemm_bs_kernel<BN, STAGES, KS, LAYOUT, PAIR>;
+    auto kern = dg::fp8_gemm_bs_kernel<BN, STAGES, KS, LAYOUT, PAIR, SPLIT>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices)
@@ -741,16 +770,53 @@ dg_status_t launch_bs(const void *A, uint64_t a_rows, const void *B, uint64_t b_
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+    attr[0].val.clusterDim.x = PAIR ? 2u : (SPLIT ? static_cast<unsigned>(p.ksplit) : 1u);
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = PAIR ? 1 : 0;
+    cfg.numAttrs = (PAIR || SPLIT) ? 1 : 0;
     if (cudaLaunchKernelEx(&cfg, kern, ta, tb, td64, tdrem, p) != cudaSuccess) {
         (void)cudaGetLastError();
         return DG_ERR_CUDA;
     }
     return DG_OK;
+}
+
+// Co-resident clusters of S CTAs of the UE8M0 split kernel (cached per
+// device, bounded by the SM cap).
+int bs_split_max_clusters(int S)
+{
+    static int cache[kMaxDevices][4] = {};  // S = 2, 4, 8 (index log2(S) - 1)
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices || S < 2 || S > 8)
+        return 0;
+    const int idx = S == 2 ? 0 : (S == 4 ? 1 : 2);
+    if (cache[dev][idx] == 0) {
+        using Cfg = dg::BsConfig<kBsSplitBN, 3, 2, false, true>;
+        auto kern = dg::fp8_gemm_bs_kernel<kBsSplitBN, 3, 2, dg::kDense, false, true>;
+        int n = 0;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) ==
+            cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(static_cast<unsigned>(S * 16), 1, 1);
+            cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+            cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess)
+                n = 0;
+        }
+        (void)cudaGetLastError();
+        cache[dev][idx] = n > 0 ? n : -1;
+    }
+    const int cap = effective_sms(dev) / S;
+    const int n = cache[dev][idx];
+    return n < 0 ? 0 : (n < cap ? n : cap);
 }
 
 template <int LAYOUT>
@@ -760,6 +826,24 @@ dg_status_t dispatch_bs(const BsChoice &c, const void *A, uint64_t a_rows, const
     p.num_nb = (p.N + c.bn - 1) / c.bn;
     p.ksplit = 1;
     p.kb_per_split = p.num_kb;
+    if constexpr (LAYOUT == dg::kDense) {
+        if (c.ksplit > 1) {
+            // one tile per cluster of ksplit CTAs; fp32 partials in the workspace
+            p.ksplit = c.ksplit;
+            p.kb_per_split = (p.num_kb + c.ksplit - 1) / c.ksplit;
+            const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
+            const size_t bytes = static_cast<size_t>(tiles) * c.ksplit * c.bn * dg::kBM * sizeof(float);
+            void *ws = nullptr;
+            const dg_status_t st = split_workspace(current_device(), bytes, &ws);
+            if (st != DG_OK)
+                return st;
+            p.ws = static_cast<float *>(ws);
+            if (c.bn == kBsSplitBN && c.stages == 3 && c.ks == 2)
+                return launch_bs<kBsSplitBN, 3, 2, LAYOUT, false, true>(A, a_rows, B, b_rows, p,
+                                                                       static_cast<int>(tiles * c.ksplit), stream);
+            return DG_ERR_UNSUPPORTED;
+        }
+    }
     if (c.pair) {
         // the pair scheduler counts 256-row pair rows
         p.num_mb = (p.num_mb + 1) / 2;
@@ -1074,10 +1158,10 @@ dg_status_t dg_fp8_gemm_nt_ue8m0(const void *A, const int32_t *sfa, const void *
     if (sms <= 0)
         return DG_ERR_CUDA;
     GemmParams p = bs_params(sfa, sfb, D, M, N, K, 1);
-    const BsChoice c = choose_bs(p.num_mb, (M + 255) / 256, N, sms);
+    const BsChoice c = choose_bs_dense(p.num_mb, (M + 255) / 256, N, p.num_kb, sms);
     if (print_configs())
-        std::fprintf(stderr, "[dg] dense ue8m0 M=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d sms=%d\n", M, N,
-                     K, c.pair ? 256 : 128, c.bn, c.stages, c.ks, sms);
+        std::fprintf(stderr, "[dg] dense ue8m0 M=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d ksplit=%d sms=%d\n",
+                     M, N, K, c.pair ? 256 : 128, c.bn, c.stages, c.ks, c.ksplit, sms);
     return dispatch_bs<dg::kDense>(c, A, static_cast<uint64_t>(M), B, static_cast<uint64_t>(N), p, sms,
                                    stream);
 }
@@ -1253,10 +1337,12 @@ int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, i
         // the UE8M0 block-scaled mode (one-CTA or pair tiles, no K split)
         const int64_t mb = static_cast<int64_t>((M + 127) / 128) * (layout == 5 ? groups : 1);
         const int64_t pr = static_cast<int64_t>((M + 255) / 256) * (layout == 5 ? groups : 1);
-        const BsChoice c = layout == 5 ? choose_bs_masked(mb, pr, N, sms) : choose_bs(mb, pr, N, sms);
+        const BsChoice c = layout == 5   ? choose_bs_masked(mb, pr, N, sms)
+                           : layout == 3 ? choose_bs_dense(mb, pr, N, K / 128 > 0 ? K / 128 : 1, sms)
+                                         : choose_bs(mb, pr, N, sms);
         return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
-                             "layout=%d BM=%d BN=%d BK=128 stages=%d ks=%d ksplit=1 pair=%d wg=1 sms=%d m_blocks=%lld n_blocks=%d ue8m0=1",
-                             layout, c.pair ? 256 : 128, c.bn, c.stages, c.ks, c.pair, sms,
+                             "layout=%d BM=%d BN=%d BK=128 stages=%d ks=%d ksplit=%d pair=%d wg=1 sms=%d m_blocks=%lld n_blocks=%d ue8m0=1",
+                             layout, c.pair ? 256 : 128, c.bn, c.stages, c.ks, c.ksplit, c.pair, sms,
                              static_cast<long long>(c.pair ? pr : mb), (N + c.bn - 1) / c.bn);
     }
     int64_t m_blocks = (M + 127) / 128;

@@ -92,15 +92,17 @@ __device__ __forceinline__ void sf_load_group(uint32_t slot, uint32_t staged_bar
     cp_async_mbar_arrive_noinc(staged_bar);
 }
 
-// BN: tile width; STAGES: ring depth; KS: 128-wide K blocks per stage (1, 2
-// or 4, so a stage never straddles a group of four K blocks); PAIR: 256-row
-// tiles on a CTA pair.
-template <int BN_, int STAGES_, int KS_, bool PAIR_>
+// BN: tile width; STAGES: ring depth; KS: 128-wide K blocks per stage; PAIR:
+// 256-row tiles on a CTA pair; SPLIT: (dense, one-CTA) the K range of each
+// tile split over the CTAs of a cluster, whose fp32 partial tiles meet in an
+// L2-resident workspace and are summed in a fixed order.
+template <int BN_, int STAGES_, int KS_, bool PAIR_, bool SPLIT_ = false>
 struct BsConfig {
     static constexpr int BN = BN_;
     static constexpr int STAGES = STAGES_;
     static constexpr int KS = KS_;
     static constexpr bool PAIR = PAIR_;
+    static constexpr bool SPLIT = SPLIT_;
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;  // rows of B this CTA loads
     static constexpr int NUM_EPI_WARPS = 4;
     static constexpr int PRODUCER_A = 4;
@@ -132,29 +134,32 @@ struct BsConfig {
     static constexpr int PIPE_BYTES = STAGES * (STAGE_A + STAGE_B) + SF_RING * SF_GROUP_BYTES;
     static constexpr int EPI_OFFSET = (PIPE_BYTES + BAR_BYTES + 1023) / 1024 * 1024;
     static constexpr int EPI_BUFS = 1024 + EPI_OFFSET + 2 * EPI_BOX_BYTES <= 232448 ? 2 : 1;
-    static constexpr int SMEM_BYTES = 1024 + EPI_OFFSET + EPI_BUFS * EPI_BOX_BYTES;
+    // (a split kernel writes its partial tile to global memory: no staging)
+    static constexpr int SMEM_BYTES = 1024 + EPI_OFFSET + (SPLIT ? 0 : EPI_BUFS * EPI_BOX_BYTES);
 
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N: multiple of 16, <= 256");
     static_assert(!PAIR || BN % 32 == 0, "a pair tile's B half must be whole 16-row TMA boxes");
     static_assert(EPI_REM % 8 == 0, "remainder box must be whole 16-byte chunks");
-    static_assert(KS == 1 || KS == 2 || KS == 4, "a stage must lie inside one group of four K blocks");
+    static_assert(KS == 1 || KS == 2 || KS == 4, "K blocks per stage");
+    static_assert(!SPLIT || (!PAIR && BN % 4 == 0), "K split: one-CTA tiles, float4 partial columns");
     static_assert(SF_COL0 % 16 == 0 && TSLOTS >= 2, "accumulators and two scale slots must fit in TMEM");
     static_assert(4 + 4 * SFB_CHUNKS <= SF_SLOT_COLS, "scale slot too small");
     static_assert(B_BYTES % 1024 == 0, "B tiles must keep 1024-byte swizzle atoms aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
-template <int BN, int STAGES, int KS, int LAYOUT, bool PAIR>
-__global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
+template <int BN, int STAGES, int KS, int LAYOUT, bool PAIR, bool SPLIT = false>
+__global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS, 1)
     fp8_gemm_bs_kernel(const __grid_constant__ CUtensorMap tmap_a,
                        const __grid_constant__ CUtensorMap tmap_b,
                        const __grid_constant__ CUtensorMap tmap_d64,
                        const __grid_constant__ CUtensorMap tmap_drem, const GemmParams p)
 {
-    using Cfg = BsConfig<BN, STAGES, KS, PAIR>;
+    using Cfg = BsConfig<BN, STAGES, KS, PAIR, SPLIT>;
     using Sched = std::conditional_t<PAIR, PairScheduler<LAYOUT>, TileScheduler<LAYOUT>>;
     static_assert(LAYOUT == kDense || LAYOUT == kContiguous || LAYOUT == kMasked,
                   "block-scaled mode: dense, contiguous and masked layouts");
+    static_assert(!SPLIT || LAYOUT == kDense, "the K split is implemented for the dense layout");
     constexpr int NACC = Cfg::NACC;
     constexpr int TSLOTS = Cfg::TSLOTS;
     constexpr int TILE_ROWS = PAIR ? kPairBM : kBM;
@@ -248,6 +253,21 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
         else
             mbar_arrive(bar_lead);
     };
+    // this CTA's K blocks [kb_lo, kb_hi) of the current tile (a K split gives
+    // each CTA of the cluster its share; a stage may then straddle two
+    // groups of four K blocks, so the scale slots go by K block)
+    auto kb_lo = [&](const Sched &sc) {
+        if constexpr (SPLIT)
+            return sc.kb_begin();
+        else
+            return 0;
+    };
+    auto kb_hi = [&](const Sched &sc) {
+        if constexpr (SPLIT)
+            return sc.kb_end();
+        else
+            return p.num_kb;
+    };
 
     if (warp == Cfg::PRODUCER_A || warp == Cfg::PRODUCER_B) {
         // ------------------------------------------------- TMA producers
@@ -260,7 +280,7 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
             const int row = is_a ? (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * TILE_ROWS +
                                        static_cast<int>(rank) * kBM
                                  : tc.g * p.N + tc.nb * BN + static_cast<int>(rank) * Cfg::B_ROWS;
-            for (int kb0 = 0; kb0 < p.num_kb; kb0 += KS) {
+            for (int kb0 = kb_lo(sched); kb0 < kb_hi(sched); kb0 += KS) {
                 if (!wait(smem_addr(empty_bar + stage), phase ^ 1, kRoleProducer, stage)) {
                     ok = false;
                     break;
@@ -322,7 +342,8 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
             const int32_t *sfb_g = p.sfb + static_cast<size_t>(tc.g) * p.num_kg * p.nbn;
             const int a_row0 = tc.mb * TILE_ROWS + static_cast<int>(rank) * kBM + lane;
             const int n_row0 = tc.nb * BN + lane;
-            for (int kg = 0; kg < p.num_kg; ++kg, ++gs) {
+            const int kg_hi = (kb_hi(sched) - 1) / 4;
+            for (int kg = kb_lo(sched) / 4; kg <= kg_hi; ++kg, ++gs) {
                 const uint32_t slot = gs % Cfg::SF_RING, sph = (gs / Cfg::SF_RING) & 1;
                 if (!wait(smem_addr(staged_empty + slot), sph ^ 1, kRoleProducer, 96 + slot)) {
                     ok = false;
@@ -344,7 +365,8 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
         uint32_t gs = 0;
         bool ok = true;
         while (ok && sched.next(tc, false)) {
-            for (int kg = 0; kg < p.num_kg; ++kg, ++gs) {
+            const int kg_hi = (kb_hi(sched) - 1) / 4;
+            for (int kg = kb_lo(sched) / 4; kg <= kg_hi; ++kg, ++gs) {
                 const uint32_t rslot = gs % Cfg::SF_RING, rph = (gs / Cfg::SF_RING) & 1;
                 const uint32_t tslot = gs % TSLOTS, tph = (gs / TSLOTS) & 1;
                 if (!wait(smem_addr(staged_full + rslot), rph, kRoleProducer, 112 + rslot) ||
@@ -390,23 +412,29 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + buf * Cfg::ACC_STRIDE;
-                for (int kb0 = 0; kb0 < p.num_kb; kb0 += KS) {
-                    const uint32_t g = gs + static_cast<uint32_t>(kb0 / 4);
-                    const uint32_t tslot = g % TSLOTS;
-                    if (!wait(smem_addr(full_bar + stage), phase, kRoleMma, stage) ||
-                        (kb0 % 4 == 0 && !wait(smem_addr(sf_full + tslot), (g / TSLOTS) & 1, kRoleMma, 24 + tslot))) {
+                const int kbl = kb_lo(sched), kbh = kb_hi(sched);
+                for (int kb0 = kbl; kb0 < kbh; kb0 += KS) {
+                    if (!wait(smem_addr(full_bar + stage), phase, kRoleMma, stage)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after_sync();
-                    const uint32_t sf_col = tmem_base + Cfg::SF_COL0 + tslot * Cfg::SF_SLOT_COLS;
-                    const bool group_done = kb0 + KS >= p.num_kb || (kb0 + KS) % 4 == 0;
-                    if (elect_one()) {
 #pragma unroll
-                        for (int q = 0; q < KS; ++q) {
-                            const int kb = kb0 + q;
-                            if (kb >= p.num_kb)
-                                break;
+                    for (int q = 0; q < KS; ++q) {
+                        const int kb = kb0 + q;
+                        if (kb >= kbh)
+                            break;
+                        // the K block's scale slot: its group's sequence number
+                        const uint32_t g = gs + static_cast<uint32_t>(kb / 4 - kbl / 4);
+                        const uint32_t tslot = g % TSLOTS;
+                        if ((kb == kbl || kb % 4 == 0) &&
+                            !wait(smem_addr(sf_full + tslot), (g / TSLOTS) & 1, kRoleMma, 24 + tslot)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint32_t sf_col = tmem_base + Cfg::SF_COL0 + tslot * Cfg::SF_SLOT_COLS;
+                        const bool group_done = kb + 1 == kbh || (kb + 1) % 4 == 0;
+                        if (elect_one()) {
                             const uint32_t byte = static_cast<uint32_t>(kb & 3);
                             const uint32_t idesc = idesc_mxf8_e4m3_ue8m0(TILE_ROWS, BN, byte);
                             const uint64_t ad =
@@ -415,7 +443,7 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
                                 b_desc0 + static_cast<uint64_t>((stage * Cfg::STAGE_B + q * Cfg::B_BYTES) >> 4);
 #pragma unroll
                             for (int j = 0; j < kBK / 32; ++j) {
-                                const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
+                                const uint32_t acc = (kb > kbl || j > 0) ? 1u : 0u;
                                 if constexpr (PAIR)
                                     mma_mxf8f6f4_bs_pair(d_tmem, ad + 2 * j, bd + 2 * j, idesc, sf_col | (byte << 30),
                                                          (sf_col + 4) | (byte << 30), acc);
@@ -423,16 +451,22 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
                                     mma_mxf8f6f4_bs(d_tmem, ad + 2 * j, bd + 2 * j, idesc, sf_col | (byte << 30),
                                                     (sf_col + 4) | (byte << 30), acc);
                             }
+                            if (group_done) {
+                                if constexpr (PAIR)
+                                    mma_commit_pair_multicast(smem_addr(sf_empty + tslot), 0x3);
+                                else
+                                    mma_commit(smem_addr(sf_empty + tslot));
+                            }
                         }
-                        if constexpr (PAIR) {
+                        __syncwarp();
+                    }
+                    if (!ok)
+                        break;
+                    if (elect_one()) {
+                        if constexpr (PAIR)
                             mma_commit_pair_multicast(smem_addr(empty_bar + stage), 0x3);
-                            if (group_done)
-                                mma_commit_pair_multicast(smem_addr(sf_empty + tslot), 0x3);
-                        } else {
+                        else
                             mma_commit(smem_addr(empty_bar + stage));
-                            if (group_done)
-                                mma_commit(smem_addr(sf_empty + tslot));
-                        }
                     }
                     __syncwarp();
                     last_bar = smem_addr(empty_bar + stage);
@@ -444,7 +478,7 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
                 }
                 if (!ok)
                     break;
-                gs += static_cast<uint32_t>(p.num_kg);
+                gs += static_cast<uint32_t>((kbh - 1) / 4 - kbl / 4 + 1);
                 if (elect_one()) {
                     if constexpr (PAIR)
                         mma_commit_pair_multicast(smem_addr(tfull_bar + buf), 0x3);
@@ -524,6 +558,19 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
                     if (lane == 0)
                         arrive_lead(tempty_lead + 8 * buf);
                 }
+                if constexpr (SPLIT) {
+                    // this split's fp32 partial of the box to the workspace,
+                    // [tile][split][BN/4][128][4]: a warp's 32 rows write 512
+                    // contiguous bytes per column quad
+                    const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
+                    float4 *dst = reinterpret_cast<float4 *>(p.ws) +
+                                  ((tile * p.ksplit + cluster_ctarank()) * (BN / 4) + cbase / 4) * kBM + row;
+#pragma unroll
+                    for (int c = 0; c < 64; c += 4)
+                        if (c < ncols)
+                            dst[(c / 4) * kBM] = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+                    continue;
+                }
                 const bool box_in = col0 + cbase < p.N;
                 if (tile_rows_ok) {
                     if (!box_in)
@@ -562,6 +609,8 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
         }
         if (threadIdx.x == 0)
             bulk_wait_group<0>();
+        if constexpr (SPLIT)
+            __threadfence();  // the partial tile is visible to the cluster's reduction
         __syncwarp();
     }
 
@@ -570,6 +619,45 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR>::THREADS, 1)
         // no CTA leaves (or frees TMEM) while its peer may still signal its
         // barriers or the leader's MMAs may still write its TMEM
         cluster_sync();
+    }
+    if constexpr (SPLIT) {
+        cluster_sync();  // every split's partial tile is in the workspace
+        // CTA `rank` sums rows [rank*128/S, (rank+1)*128/S) of the tile over
+        // the S partials in split order (a fixed order: results do not
+        // depend on timing) and rounds them to bf16.
+        const int S = p.ksplit;
+        const uint32_t rank_s = cluster_ctarank();
+        Sched sched(p);
+        TileCoord tc;
+        if (sched.next(tc, false)) {
+            const int rows_per = kBM / S;
+            constexpr int C4 = BN / 4;
+            const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
+            const float4 *src0 = reinterpret_cast<const float4 *>(p.ws) + tile * S * C4 * kBM;
+            for (int it = threadIdx.x; it < rows_per * C4; it += Cfg::THREADS) {
+                const int lr = it % rows_per;  // rows fastest: contiguous reads
+                const int c4 = it / rows_per;
+                const int r = static_cast<int>(rank_s) * rows_per + lr;
+                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int src = 0; src < S; ++src) {
+                    const float4 w = __ldcg(src0 + (static_cast<size_t>(src) * C4 + c4) * kBM + r);
+                    sum.x += w.x;
+                    sum.y += w.y;
+                    sum.z += w.z;
+                    sum.w += w.w;
+                }
+                const int grow = tc.mb * kBM + r;
+                const int gcol = tc.nb * BN + c4 * 4;
+                if (grow < p.M && gcol < p.N) {
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
+                    uint2 u;
+                    u.x = *reinterpret_cast<uint32_t *>(&h0);
+                    u.y = *reinterpret_cast<uint32_t *>(&h1);
+                    *reinterpret_cast<uint2 *>(p.D + static_cast<size_t>(grow) * p.N + gcol) = u;
+                }
+            }
+        }
     }
     if (warp == Cfg::MMA_WARP) {
         tc_fence_after_sync();

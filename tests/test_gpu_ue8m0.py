@@ -143,6 +143,24 @@ def test_dense_ue8m0_deterministic(dg, oracle_mod, family):
     assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (64, 1024, 4096),     # 8 tiles, 4 K blocks per split
+    (100, 4096, 3200),    # 25 K blocks: 7 per split, stages straddle K-block groups
+    (200, 2112, 1024),    # two m-blocks, 2 K blocks per split
+])
+def test_dense_ue8m0_k_split(dg, oracle_mod, M, N, K):
+    """Decode-shaped problems split each tile's K range over a cluster; the
+    fp32 partials meet in the workspace and are summed in a fixed order."""
+    plan = _plan(dg, 3, M, N, K)
+    assert int(plan["ksplit"]) > 1, plan
+    p = gi.dense_problem(M, N, K, seed_a=7000 + M, seed_b=8000 + N, ue8m0=True)
+    got, _ = _dense(dg, oracle_mod, p)
+    _, ref = oracle_mod.gemm_nt(p["A"], p["sA"], p["B"], p["sB"], want_f64=False)
+    assert_close(got, ref, f"ue8m0 split {M}x{N}x{K}")
+    again, _ = _dense(dg, oracle_mod, p)
+    assert np.array_equal(got, again)  # fixed reduction order
+
+
 def test_dense_decode_ue8m0_full(dg, oracle_mod):
     """The decode-shaped benchmark problem (128 x 2112 x 7168), whole output."""
     p = gi.make_workload("dense_decode", ue8m0=True)
@@ -264,3 +282,44 @@ def test_transform_extreme_exponents(dg, oracle_mod):
     out = dg.dg_transform_sf_ue8m0(torch.from_numpy(s).to(dev), 51, mn_major=False)
     assert dg.dg_get_device_status() == 0
     assert np.array_equal(out.cpu().numpy(), oracle_mod.pack_ue8m0(s))
+
+
+# ------------------------------------------------------ bounded waits
+
+@pytest.mark.parametrize("M,N,K,fam,first_ctas", [
+    (1024, 4096, 4096, 1, 1),   # one-CTA tiles
+    (2048, 4096, 4096, 2, 2),   # CTA pairs
+])
+def test_ue8m0_wait_timeout_is_reported_and_the_context_survives(dg, oracle_mod, M, N, K, fam, first_ctas):
+    """With the stall injection hook the first CTA (or pair) never receives
+    its operands: every wait of the block-scaled kernel is bounded, so it
+    records DG_ERR_TIMEOUT, drains its scale copies, frees TMEM and returns,
+    and the next call on the same buffers is correct."""
+    p = gi.dense_problem(M, N, K, seed_a=75, seed_b=76, ue8m0=True)
+    dg.dg_set_tile_family(fam)
+    dg.dg_set_wait_timeout_ns(20_000_000)
+    dg.dg_set_stall_injection(True)
+    try:
+        assert _plan(dg, 3, M, N, K)["pair"] == str(fam - 1)
+        dev = torch.device("cuda")
+        A = torch.from_numpy(p["A"]).to(dev)
+        B = torch.from_numpy(p["B"]).to(dev)
+        sfa, sfb = _packed(dg, oracle_mod, p["sA"], p["sB"])
+        D = torch.full((M, N), SENTINEL, dtype=torch.int16, device=dev).view(torch.bfloat16)
+        dg.dg_fp8_gemm_nt_ue8m0(A, sfa, B, sfb, D)
+        st, word = dg.dg_get_device_status_detail()
+    finally:
+        dg.dg_set_stall_injection(False)
+        dg.dg_set_wait_timeout_ns(0)
+    try:
+        assert st == 5, f"status {st}, word {word:#x}"
+        assert (word >> 8) & 0xF in (1, 2, 3)  # scale writers, MMA or epilogue
+        assert word >> 20 < first_ctas          # in the stalled CTA (or pair)
+        assert dg.dg_get_device_status() == 5   # read and cleared
+        assert dg.dg_get_device_status() == 0
+        dg.dg_fp8_gemm_nt_ue8m0(A, sfa, B, sfb, D)
+        assert dg.dg_get_device_status() == 0
+    finally:
+        dg.dg_set_tile_family(dg.DG_TILES_AUTO)
+    _, ref = oracle_mod.gemm_nt(p["A"], p["sA"], p["B"], p["sB"], want_f64=False)
+    assert_close(bits(D), ref, f"ue8m0 after a timeout, {M}x{N}x{K}")
