@@ -261,7 +261,11 @@ dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, const void *B
  * m_indices, masked_m, the validation rules and the device status behaviour
  * are those of dg_fp8_gemm_nt, dg_fp8_grouped_gemm_contiguous and
  * dg_fp8_grouped_gemm_masked.  These calls run one-CTA tiles (128 x BN, BN
- * in {128, 160, 192, 224}) and allocate nothing.
+ * in {128, 160, 192, 224}) or CTA-pair tiles (256 x BN); a dense problem with
+ * too few tiles to fill the GPU splits K over a cluster of CTAs and uses the
+ * library-owned split workspace described above (same rules: make the first
+ * such call before any stream capture, and do not overlap such calls on the
+ * GPU).  Everything else allocates nothing.
  */
 dg_status_t dg_fp8_gemm_nt_ue8m0(const void *A, const int32_t *sfa, const void *B,
                                  const int32_t *sfb, void *D, int M, int N, int K,
