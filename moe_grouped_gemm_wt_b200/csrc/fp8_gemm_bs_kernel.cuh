@@ -45,6 +45,10 @@
 // commits arrive on both CTAs' barriers (multicast arrive, not a data copy).
 // Per SM and K block the operand bytes then drop from (128 + BN) * 128 to
 // (128 + BN/2) * 128.
+// Dense problems with too few tiles to fill the GPU (decode shapes) split
+// each tile's K range over a cluster of CTAs instead: each writes its fp32
+// partial tile to an L2-resident workspace, and after a cluster barrier each
+// sums a slice of the tile's rows over the partials in a fixed order.
 //
 // Waits are bounded: a wait that runs out records DG_ERR_TIMEOUT, raises the
 // CTA's (and on a pair its peer's) abort flag and every role leaves; copies

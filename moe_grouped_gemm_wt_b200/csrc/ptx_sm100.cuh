@@ -248,20 +248,6 @@ __device__ __forceinline__ void cp_async_4_zfill(uint32_t dst, const void *src, 
                  : "memory");
 }
 
-// Closes this thread's current group of cp.async copies.
-__device__ __forceinline__ void cp_async_commit_group()
-{
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// Waits until at most N of this thread's most recent cp.async groups are
-// still pending.
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group()
-{
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 __device__ __forceinline__ uint4 ld_shared_v4u(uint32_t addr)
 {
     uint4 v;
