@@ -666,9 +666,12 @@ struct BsChoice {
 };
 
 // The dense decode plan of the UE8M0 mode: problems with too few tiles to
-// fill the GPU split each 128 x 144 tile's K range over a cluster of S CTAs
-// (S = 8, 4 or 2: the largest that leaves every split two K blocks and keeps
-// all of the grid's clusters co-resident).
+// fill the GPU and a long K range (at least 16 K blocks: below that the
+// cluster barrier and the reduction cost more than the split saves, e.g.
+// 16.4 vs 11.1 us on 128 x 256 x 512) split each 128 x 144 tile's K range
+// over a cluster of S CTAs (S = 8, 4 or 2: the largest that leaves every
+// split two K blocks and keeps all of the grid's clusters co-resident).
+constexpr int kBsSplitMinKb = 16;
 constexpr int kBsSplitBN = 144;
 int bs_split_max_clusters(int S);
 constexpr BsChoice kBsChoices[] = {
@@ -707,7 +710,7 @@ BsChoice choose_bs_dense(int64_t m_blocks, int64_t pair_rows, int N, int num_kb,
     if (forced_block_n() > 0 || forced_pair() == 1)
         return c;
     const int64_t tiles = m_blocks * ((N + c.bn - 1) / c.bn);
-    if (c.pair || tiles * 2 > sms)
+    if (c.pair || tiles * 2 > sms || num_kb < kBsSplitMinKb)
         return c;
     const int64_t split_tiles = m_blocks * ((N + kBsSplitBN - 1) / kBsSplitBN);
     for (int S = 8; S >= 2; S /= 2) {

@@ -146,7 +146,7 @@ def test_dense_ue8m0_deterministic(dg, oracle_mod, family):
 @pytest.mark.parametrize("M,N,K", [
     (64, 1024, 4096),     # 8 tiles, 4 K blocks per split
     (100, 4096, 3200),    # 25 K blocks: 7 per split, stages straddle K-block groups
-    (200, 2112, 1024),    # two m-blocks, 2 K blocks per split
+    (200, 1024, 2048),    # two m-blocks, 16 K blocks: 2 or 4 per split
 ])
 def test_dense_ue8m0_k_split(dg, oracle_mod, M, N, K):
     """Decode-shaped problems split each tile's K range over a cluster; the
