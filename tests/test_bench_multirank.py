@@ -106,3 +106,29 @@ def test_expert_shards_partition_the_grouped_problems(oracle_mod, world):
         got.append(oracle_mod.grouped_masked(q["A"], q["sA"], q["B"], q["sB"], q["masked_m"],
                                              np.full((q["G"], 200, 144), SENT, np.uint16))[1])
     assert np.array_equal(np.concatenate(got), fullm)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_expert_shards_of_a_ue8m0_problem_keep_the_mode(oracle_mod, world):
+    """`bench.py --scales ue8m0` shards grouped problems the same way: the
+    shards keep the mode, and their (power-of-two) scales pack into UE8M0
+    words and back unchanged."""
+    import sys
+    import numpy as np
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import bench
+    import dg_inputs as gi
+
+    for p in (gi.contiguous_problem([100, 300, 37, 128], 144, 512, seed_a=95, seed_b=96, ue8m0=True),
+              gi.masked_problem(4, 200, 144, 512, masked_m=[0, 200, 77, 3], seed_a=97, seed_b=98,
+                                ue8m0=True)):
+        p["ue8m0"] = True
+        for r in range(world):
+            q = bench.shard_experts(p, r, world)
+            assert q["ue8m0"]
+            if q["G"] == 0:
+                continue
+            for s in (q["sA"], q["sB"]):
+                nkb = s.shape[-1]
+                assert np.array_equal(oracle_mod.unpack_ue8m0(oracle_mod.pack_ue8m0(s), nkb), s)
