@@ -149,6 +149,27 @@ def test_ue8m0_describe_config(lib):
     assert lib.dg_describe_config(6, 128, 256, 512, 1, buf, 256) == -1
 
 
+def test_ue8m0_planner_under_an_sm_cap(lib):
+    """The UE8M0 planner (host only): with 16 SMs, 16 one-CTA 128x224 tiles or
+    8 pair tiles of 256x224 fill the GPU in one wave, and the pair family
+    (half the B traffic per SM) wins; the masked layout takes the one-CTA
+    128-column tile; a forced family is honoured."""
+    buf = ctypes.create_string_buffer(256)
+    desc = lambda *a: (lib.dg_describe_config(*a, buf, 256), dict(kv.split("=") for kv in buf.value.decode().split()))[1]
+    assert lib.dg_set_num_sms(16) == 0
+    try:
+        d = desc(3, 2048, 224, 512, 1)
+        assert (d["BN"], d["pair"], d["BM"]) == ("224", "1", "256"), d
+        d = desc(5, 100, 4096, 7168, 16)
+        assert (d["BN"], d["pair"], d["stages"]) == ("128", "0", "3"), d
+        assert lib.dg_set_tile_family(1) == 0  # one-CTA tiles only
+        d = desc(3, 2048, 224, 512, 1)
+        assert (d["BN"], d["pair"]) == ("224", "0"), d
+    finally:
+        lib.dg_set_tile_family(0)
+        lib.dg_set_num_sms(0)
+
+
 def test_sm_fill_example_from_pages(lib):
     """The unaligned-block-size example of the DeepGEMM article (lqnn.cn,
     section 非对齐块大小): M=256, N=7168 on 132 SMs -- 128x128 tiles occupy
