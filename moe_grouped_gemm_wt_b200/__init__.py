@@ -433,8 +433,10 @@ def dg_fp8_gemm_nt_ue8m0(A, sfa, B, sfb, D, stream=None) -> None:
     psa = _dev(sfa, "sfa", _I32, 2)
     if tuple(sfa.shape) != (_ng(K), get_tma_aligned_size(M, 4)):
         raise ValueError(f"sfa must be [ceil(K/512), M_pad] = {(_ng(K), get_tma_aligned_size(M, 4))}")
-    psb = _dev(sfb, "sfb", _I32, sfb.dim() if isinstance(sfb, torch.Tensor) and sfb.dim() in (2, 3) else 2)
-    if tuple(sfb.shape)[-2:] != (_ng(K), (N + 127) // 128) or (sfb.dim() == 3 and sfb.shape[0] != 1):
+    if isinstance(sfb, torch.Tensor) and sfb.dim() == 3 and sfb.shape[0] == 1:
+        sfb = sfb[0]  # a one-group weight-scale array
+    psb = _dev(sfb, "sfb", _I32, 2)
+    if tuple(sfb.shape) != (_ng(K), (N + 127) // 128):
         raise ValueError("sfb must be [ceil(K/512), ceil(N/128)]")
     pd = _dev(D, "D", _BF16, 2)
     if tuple(D.shape) != (M, N):
