@@ -10,7 +10,9 @@
  * and one per 128x128 block of B.  Each 128-wide K block is contracted on the
  * tensor cores and its partial is then promoted into an fp32 accumulator on
  * the CUDA cores as acc += (sA*sB) * partial.  D is bf16, rounded to nearest
- * even once at the end.
+ * even once at the end.  A separately declared UE8M0 mode (the *_ue8m0 calls
+ * below) takes power-of-two scales packed four to an int32 and lets the
+ * tensor core apply them (block-scaled MMA, fp32 accumulation in TMEM).
  *
  * Sources (the DeepGEMM pages):
  *  - "DeepGEMM: kernel FP8 GEMM sach va hieu qua nho scaling chi tiet"
