@@ -24,7 +24,8 @@ Parity status of each function (what pins it is listed in the tests):
                                 (exact), C alone (A = 0), the closed form
                                 C + float64 matmul, numpy's double->float32
   grouped_contiguous / masked   pinned: per-group dense results, placement,
-                                untouched padding / masked rows
+                                untouched padding / masked rows, malformed
+                                contiguous blocks written by hand-listed rows
   fp32_promotion_sampled        analysis aid (not a reference), pinned against
                                 a float32 re-computation on small cases
   ue8m0_value / ue8m0_from_scale  pinned: every code vs Python's exact 2.0**k,
@@ -262,7 +263,8 @@ def fp32_promotion_sampled(A, sA, B, sB, rows, cols):
 
 def grouped_contiguous(A, sA, B, sB, m_indices, D16_init, want_f64=False):
     """Contiguous grouped GEMM.  D16_init ([M_total][N] uint16) is copied and
-    only rows with a valid group index are overwritten."""
+    only rows whose group index is valid and equals the index of the first
+    row of their 128-row block are overwritten."""
     A, B, sA, sB = _u8(A), _u8(B), _f32(sA), _f32(sB)
     m_indices = np.ascontiguousarray(m_indices, dtype=np.int32)
     M, K = A.shape

@@ -312,9 +312,15 @@ int dgo_gemm_nt_sampled(const uint8_t *A, const float *sA, const uint8_t *B,
 
 /* --------------------------------------------------- contiguous grouped */
 
-/* Contiguous grouped layout: rows of all groups concatenated along M.
- * Row m belongs to group g = m_indices[m]; it uses B_g and sB_g.  A row whose
- * index is outside [0, G) (padding) is not written.
+/* Contiguous grouped layout: rows of all groups concatenated along M, each
+ * group's segment starting on a multiple of DGO_BLOCK rows (the segments are
+ * aligned to the M block), so every aligned block of DGO_BLOCK rows belongs
+ * to the one group named by its first row.  Row m is written, with B_g and
+ * sB_g, when g = m_indices[m] lies in [0, G) and equals the index of the
+ * first row of its block.  Every other row is not written: padding rows
+ * (negative index), the rows of a block whose first row is padding or out of
+ * range, and rows whose index disagrees with their block's first row (input
+ * that breaks the alignment rule; see dgo_check_contiguous_alignment).
  * A: [M_total][K], sA: [M_total][K/128], B: [G][N][K],
  * sB: [G][ceil(N/128)][K/128], D: [M_total][N]. */
 int dgo_grouped_contiguous(const uint8_t *A, const float *sA, const uint8_t *B,
@@ -330,7 +336,7 @@ int dgo_grouped_contiguous(const uint8_t *A, const float *sA, const uint8_t *B,
 #pragma omp parallel for schedule(dynamic, 1)
     for (int m = 0; m < M_total; ++m) {
         int g = m_indices[m];
-        if (g < 0 || g >= G)
+        if (g < 0 || g >= G || g != m_indices[(m / DGO_BLOCK) * DGO_BLOCK])
             continue;
         const uint8_t *Bg = B + (int64_t)g * N * K;
         const float *sBg = sB + (int64_t)g * nbn * nkb;

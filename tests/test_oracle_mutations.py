@@ -51,6 +51,9 @@ MUTATIONS = {
     "UE8M0 scale rounded down instead of up": (
         "    return m == 0.5 ? x : ldexp(1.0, ex);",
         "    return m == 0.5 ? x : ldexp(1.0, ex - 1);"),
+    "contiguous: row's own index instead of its block's first-row index": (
+        "        if (g < 0 || g >= G || g != m_indices[(m / DGO_BLOCK) * DGO_BLOCK])",
+        "        if (g < 0 || g >= G)"),
     "UE8M0 packing byte order reversed": (
         "                word |= (uint32_t)code << (8 * j);",
         "                word |= (uint32_t)code << (8 * (3 - j));"),
@@ -81,6 +84,8 @@ def _build_variant(tmp_path, old, new):
     lib.dgo_ue8m0_ceil_pow2.argtypes = [ctypes.c_double]
     lib.dgo_pack_ue8m0.restype = I
     lib.dgo_pack_ue8m0.argtypes = [P, I, I, P]
+    lib.dgo_grouped_contiguous.restype = I
+    lib.dgo_grouped_contiguous.argtypes = [P, P, P, P, P, I, I, I, I, P, P]
     return lib
 
 
@@ -165,6 +170,21 @@ def _pins_pass(lib) -> bool:
         return False
     want = np.array([[0x827E807F, 0x7F7F7F7D], [0x7F7F7F84, 0x7F7F7F7F]], dtype=np.uint32)
     if not np.array_equal(words.view(np.uint32), want):
+        return False
+    # contiguous placement: a block belongs to the group of its first row;
+    # hand-listed rows written (rows 0..99 and 256..383), all others untouched
+    pc = gi.contiguous_problem([384], 32, 128, seed_a=31, seed_b=32)
+    idx = np.full(384, -1, np.int32)
+    idx[0:100], idx[100:110], idx[140:200], idx[256:384] = 0, 1, 1, 0
+    b2 = np.ascontiguousarray(np.concatenate([pc["B"], pc["B"]]))
+    sb2 = np.ascontiguousarray(np.concatenate([pc["sB"], pc["sB"]]))
+    c16 = np.full((384, 32), 0x7FC1, np.uint16)
+    if lib.dgo_grouped_contiguous(_ptr(np.ascontiguousarray(pc["A"])), _ptr(np.ascontiguousarray(pc["sA"])),
+                                  _ptr(b2), _ptr(sb2), _ptr(idx), 384, 32, 128, 2, None, _ptr(c16)) != 0:
+        return False
+    written = np.zeros(384, bool)
+    written[0:100] = written[256:384] = True
+    if not (np.all(c16[~written] == 0x7FC1) and np.all(c16[written] != 0x7FC1)):
         return False
     return True
 

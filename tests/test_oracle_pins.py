@@ -307,6 +307,40 @@ def test_contiguous_alignment_checker(oracle_mod):
     assert oracle_mod.check_contiguous_alignment(idx) == -1
 
 
+def test_contiguous_malformed_blocks_written_by_block_rule(oracle_mod):
+    """Segments are aligned to the 128-row M block, so a block belongs to the
+    group of its first row.  Hand-built blocks that break the rule: the rows
+    listed below (and only they) are written, each equal to the dense GEMM
+    of its group; every other row keeps the sentinel."""
+    N, K, G = 144, 256, 2
+    M = 5 * 128
+    p = gi.contiguous_problem([M], N, K, seed_a=73, seed_b=74)
+    rng = np.random.default_rng(75)
+    B = np.stack([p["B"][0], rng.permutation(p["B"][0])])
+    sB = np.stack([p["sB"][0], p["sB"][0] * 0.5])
+    idx = np.full(M, -1, np.int32)
+    idx[0:100] = 0        # block 0: group 0, then a mid-block change to group 1
+    idx[100:110] = 1
+    idx[140:200] = 1      # block 1: first row padding, later rows valid
+    idx[256:384] = 1      # block 2: well formed
+    idx[384:512] = 5      # block 3: group out of range
+    idx[512:520] = 0      # block 4: group 0, then a row with an out-of-range index
+    idx[520] = 7
+    idx[521:600] = 0
+    init = np.full((M, N), SENTINEL, np.uint16)
+    _, d16 = oracle_mod.grouped_contiguous(p["A"], p["sA"], B, sB, idx, init)
+    written = {0: list(range(0, 100)) + list(range(512, 520)) + list(range(521, 600)),
+               1: list(range(256, 384))}
+    for g, rows in written.items():
+        rows = np.asarray(rows)
+        _, ref = oracle_mod.gemm_nt(p["A"][rows], p["sA"][rows], B[g], sB[g])
+        assert np.array_equal(d16[rows], ref), f"group {g}"
+    untouched = np.setdiff1d(np.arange(M), np.concatenate([np.asarray(r) for r in written.values()]))
+    assert untouched.size == M - 100 - 8 - 79 - 128
+    assert np.all(d16[untouched] == SENTINEL)
+    assert oracle_mod.check_contiguous_alignment(idx) == 100
+
+
 def test_masked_equals_per_group_dense_and_leaves_rest(oracle_mod):
     G, max_m, N, K = 3, 160, 144, 256
     masked_m = np.array([1, 160, 0], np.int32)
