@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
     const int lane = threadIdx.x % 32;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     const bool leader = rank == 0;
+    stamp_start(p);
 
     if (warp == Cfg::PRODUCER_A && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -513,6 +514,17 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
             // a warp that gave up takes the others with it (no warp may be
             // left waiting at a later named barrier)
             if (!named_barrier_and(1, 128, ok)) {
+                if constexpr (SPLIT) {
+                    // this split has no partial: NaN in its workspace slot,
+                    // so the cluster's sums show the failure instead of
+                    // adding a stale partial left there by an earlier call
+                    const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
+                    float4 *dst = reinterpret_cast<float4 *>(p.ws) +
+                                  (tile * p.ksplit + cluster_ctarank()) * (BN / 4) * kBM + row;
+                    const float nan = __int_as_float(0x7FC00000);
+                    for (int c4 = 0; c4 < BN / 4; ++c4)
+                        dst[c4 * kBM] = make_float4(nan, nan, nan, nan);
+                }
                 ok = false;
                 break;
             }
@@ -524,10 +536,12 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
                 row_ok = m_local < p.M;
             } else if constexpr (LAYOUT == kContiguous) {
                 row_ok = false;
+                // computed when the row's index is this visit's group and
+                // the group of its own 128-row block (its first row's)
                 const int block_g = m_half < p.M ? __ldg(p.m_indices + m_half) : -1;
                 if (m_local < p.M && block_g >= 0) {
                     const int idx = __ldg(p.m_indices + m_local);
-                    row_ok = idx == tc.g;
+                    row_ok = idx == tc.g && idx == block_g;
                     if (idx >= 0 && idx != block_g)
                         record_status(kCodeBadGroup, kRolePromote, 1);
                 }
@@ -663,6 +677,7 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
             }
         }
     }
+    stamp_end(p);
     if (warp == Cfg::MMA_WARP) {
         tc_fence_after_sync();
         if constexpr (PAIR)

@@ -106,7 +106,26 @@ struct GemmParams {
     const int32_t *sfb;  // [G][num_kg][nbn]
     int sfa_ld;          // padded row count of the packed LHS scales
     int num_kg;          // ceil(num_kb / 4)
+    // Launch timing (dg_set_timing_stamps): when set, stamps[0] takes the
+    // earliest CTA start and stamps[1] the latest CTA end (%globaltimer, ns).
+    unsigned long long *stamps;
 };
+
+// Launch-timing stamps: thread 0 of each CTA folds its start and end time
+// into the caller's pair (atomicMin / atomicMax, one each per CTA).
+__device__ __forceinline__ void stamp_start(const GemmParams &p)
+{
+    if (p.stamps != nullptr && threadIdx.x == 0)
+        atomicMin(p.stamps, static_cast<unsigned long long>(global_timer_ns()));
+}
+__device__ __forceinline__ void stamp_end(const GemmParams &p)
+{
+    if (p.stamps != nullptr) {
+        __syncthreads();
+        if (threadIdx.x == 0)
+            atomicMax(p.stamps + 1, static_cast<unsigned long long>(global_timer_ns()));
+    }
+}
 
 // Row segment of an fp32 output: drow[c] = acc[c] for the 4-float groups of
 // this thread's row that lie inside N.
@@ -144,6 +163,20 @@ constexpr int kBK = 128;
 struct TileCoord {
     int g, mb, nb;
 };
+
+// Contiguous layout: the segments are aligned to the 128-row M block, so a
+// block whose first row is padding must hold padding only.  True when any
+// row of the block [row0, row0 + 128) carries a group index (a malformed
+// block: it is skipped and its rows stay untouched, but it is flagged).
+// Run by one thread, only for blocks whose first row is padding.
+__device__ __forceinline__ bool padding_block_has_rows(const int32_t *m_indices, int row0)
+{
+    int any = 0;
+#pragma unroll 8
+    for (int r = 1; r < kBM; ++r)
+        any |= __ldg(m_indices + row0 + r) >= 0 ? 1 : 0;
+    return any != 0;
+}
 
 // Enumerates this CTA's tiles: t = blockIdx.x, blockIdx.x + gridDim.x, ...
 // Every role runs its own copy and sees the same sequence.
@@ -238,8 +271,13 @@ struct TileScheduler {
                 tc.g = 0;
                 if constexpr (LAYOUT == kContiguous) {
                     const int g = __ldg(p.m_indices + tc.mb * kBM);
-                    if (g < 0)
-                        continue;  // padding block: rows stay untouched
+                    if (g < 0) {
+                        // padding block: rows stay untouched (flagged if
+                        // any of its rows carries a group index)
+                        if (report && tc.nb == 0 && padding_block_has_rows(p.m_indices, tc.mb * kBM))
+                            record_status(kCodeBadGroup, kRoleSched, 0);
+                        continue;
+                    }
                     if (g >= p.G) {
                         if (report)
                             record_status(kCodeBadGroup, kRoleSched, 0);
@@ -295,7 +333,7 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
 // BN: tile width; STAGES: shared-memory ring depth; KS: 128-wide K blocks per
 // stage (one 3-D TMA box per operand carries all KS blocks -- the TMA engine
 // costs a roughly fixed time per instruction, so bigger boxes move more).
-template <int BN_, int STAGES_, int KS_, bool SPLIT_ = false, bool COLSCALE_ = false>
+template <int BN_, int STAGES_, int KS_, bool SPLIT_ = false, bool COLSCALE_ = false, int NWG_ = 2>
 struct KernelConfig {
     // COLSCALE: one B scale per column and K block (the K-grouped layout)
     // instead of one per 128x128 block.
@@ -307,14 +345,16 @@ struct KernelConfig {
     // through an L2-resident workspace and are summed by the cluster instead
     // of being TMA-stored.
     static constexpr bool SPLIT = SPLIT_;
-    // Two promotion warpgroups split the tile's columns; thread t of each
-    // owns tile row t.
-    static constexpr int NUM_WG = 2;
+    // NUM_WG promotion warpgroups split the tile's columns; thread t of each
+    // owns tile row t.  Four (the K-split decode tile) halve each thread's
+    // columns and double the warps that hide the TMEM-load latency.
+    static constexpr int NUM_WG = NWG_;
     static constexpr int BN_WG = BN / NUM_WG;
-    // TMEM is read in rounds of at most RMAX columns: a warpgroup with at
-    // most 64 columns pulls its whole partial in one round and frees the
-    // buffer before any arithmetic.
-    static constexpr int RMAX = BN_WG <= 64 ? BN_WG : 32;
+    // TMEM is read in rounds of at most RMAX columns: a warpgroup whose
+    // columns fit beside its accumulator in registers (64, or 40 with four
+    // warpgroups and their smaller register budget) pulls its whole partial
+    // in one round and frees the buffer before any arithmetic.
+    static constexpr int RMAX = BN_WG <= (NUM_WG >= 4 ? 40 : 64) ? BN_WG : 32;
     static constexpr int NUM_PROMO_WARPS = 4 * NUM_WG;
     static constexpr int PRODUCER_WARP = NUM_PROMO_WARPS;
     static constexpr int MMA_WARP = NUM_PROMO_WARPS + 1;
@@ -349,7 +389,10 @@ struct KernelConfig {
         1024 /*align slack*/ + EPI_OFFSET + (SPLIT ? 0 : NUM_WG * EPI_BUFS * EPI_WG_BYTES);
 
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128: multiple of 16, <= 256");
-    static_assert(BN_WG % 8 == 0, "promotion columns per warpgroup must be a multiple of 8");
+    static_assert(BN % NUM_WG == 0 && BN_WG % 4 == 0, "promotion columns per warpgroup: a multiple of 4");
+    static_assert(BN_WG % 8 == 0 || (SPLIT && !COLSCALE && BN_WG == RMAX),
+                  "a column count that is not a multiple of 8 is read in one round and split-reduced");
+    static_assert(NUM_WG * 4 + 2 <= 32 && NUM_WG <= 14, "warps per CTA; named barriers 1..NUM_WG");
     static_assert(BN_WG <= 128, "a warpgroup's columns must span at most two 128-wide sB blocks");
     static_assert(NBUF >= 2, "double-buffered TMEM at least");
     static_assert(B_BYTES % 1024 == 0, "B tiles must keep 1024-byte swizzle atoms aligned");
@@ -364,12 +407,19 @@ struct KernelConfig {
 template <int COLS>
 __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *r)
 {
+    static_assert(COLS % 4 == 0, "TMEM loads of whole 4-column groups");
 #pragma unroll
-    for (int q = 0; q < COLS; q += 16) {
-        if (q + 16 <= COLS)
+    for (int q = 0; q < COLS;) {
+        if (q + 16 <= COLS) {
             tmem_ld_32x32b_x16(taddr + q, *reinterpret_cast<uint32_t(*)[16]>(r + q));
-        else
+            q += 16;
+        } else if (q + 8 <= COLS) {
             tmem_ld_32x32b_x8(taddr + q, *reinterpret_cast<uint32_t(*)[8]>(r + q));
+            q += 8;
+        } else {
+            tmem_ld_32x32b_x4(taddr + q, *reinterpret_cast<uint32_t(*)[4]>(r + q));
+            q += 4;
+        }
     }
 }
 
@@ -394,14 +444,14 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float *v)
 // only).  Its stage tile is then loaded as 2-D TMA boxes of 128 M (or N)
 // bytes by 128*KS K rows (B: one box per 128 columns, BN % 128 == 0) and
 // described to the MMA as an MN-major 128-byte-swizzled operand.
-template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false>
-__global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped>::THREADS, 1)
+template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false, int NWG = 2>
+__global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped, NWG>::THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d64,
                     const __grid_constant__ CUtensorMap tmap_drem, const GemmParams p)
 {
-    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped>;
+    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped, NWG>;
     static_assert(!SPLIT || LAYOUT == kDense, "K split is implemented for the dense layout");
     static_assert((!A_MN && !B_MN) || LAYOUT == kDense || LAYOUT == kKGrouped,
                   "MN-major operands are implemented for the dense and K-grouped layouts");
@@ -430,6 +480,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
+    stamp_start(p);
 
     if (warp == Cfg::PRODUCER_WARP && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -747,6 +798,20 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
                             if (lane == 0)
                                 mbar_arrive(smem_addr(tempty_bar + buf));
                         }
+                        if constexpr (BN_WG % 8 != 0) {
+                            // columns in groups of 4 (one round, per-block
+                            // scales): a warpgroup starting at 4 mod 8 can
+                            // meet the 128-column scale boundary inside an
+                            // 8-column group
+#pragma unroll
+                            for (int g4 = 0; g4 < RMAX; g4 += 4) {
+                                const float sc = (c0 + g4 >= boundary) ? s_hi[q] : s_lo[q];
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    acc[c0 + g4 + i] = fmaf(__uint_as_float(r[g4 + i]), sc, acc[c0 + g4 + i]);
+                            }
+                            continue;
+                        }
 #pragma unroll
                         for (int g8 = 0; g8 < RMAX; g8 += 8) {
                             if (whole || g8 < TAIL) {
@@ -784,15 +849,18 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
             if constexpr (SPLIT) {
                 // K split: this split's fp32 partial tile goes to the
                 // workspace as [column quad][row] float4s, so the 32 rows of
-                // a warp write 512 contiguous bytes per store.
-                if (ok) {
-                    const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
-                    float4 *dst = reinterpret_cast<float4 *>(p.ws) +
-                                  ((tile * p.ksplit + cluster_ctarank()) * (BN / 4) + wg * (BN_WG / 4)) * kBM + row;
+                // a warp write 512 contiguous bytes per store.  A warp that
+                // gave up on a wait writes NaN instead: the cluster's sums
+                // for its columns then show the failure rather than add a
+                // stale partial left in the workspace by an earlier call.
+                const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
+                float4 *dst = reinterpret_cast<float4 *>(p.ws) +
+                              ((tile * p.ksplit + cluster_ctarank()) * (BN / 4) + wg * (BN_WG / 4)) * kBM + row;
+                const float nan = __int_as_float(0x7FC00000);
 #pragma unroll
-                    for (int c = 0; c < BN_WG; c += 4)
-                        dst[(c / 4) * kBM] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-                }
+                for (int c = 0; c < BN_WG; c += 4)
+                    dst[(c / 4) * kBM] = ok ? make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3])
+                                            : make_float4(nan, nan, nan, nan);
                 continue;
             }
             // A warpgroup stores its 128 rows with whole-tile TMA boxes when
@@ -894,14 +962,16 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
         TileScheduler<LAYOUT> sched(p);
         TileCoord tc;
         if (sched.next(tc, false)) {
-            const int rows_per = kBM / S;
+            // rows [r0, r1) of the tile: S need not divide 128
+            const int r0 = static_cast<int>(rank) * kBM / S;
+            const int rows_per = (static_cast<int>(rank) + 1) * kBM / S - r0;
             constexpr int C4 = BN / 4;
             const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
             const float4 *src0 = reinterpret_cast<const float4 *>(p.ws) + tile * S * C4 * kBM;
             for (int it = threadIdx.x; it < rows_per * C4; it += Cfg::THREADS) {
                 const int lr = it % rows_per;  // rows fastest: contiguous reads
                 const int c4 = it / rows_per;
-                const int r = static_cast<int>(rank) * rows_per + lr;
+                const int r = r0 + lr;
                 float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int src = 0; src < S; ++src) {
                     const float4 v = __ldcg(src0 + (static_cast<size_t>(src) * C4 + c4) * kBM + r);
@@ -929,6 +999,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
             }
         }
     }
+    stamp_end(p);
     if (warp == Cfg::MMA_WARP) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);

@@ -100,7 +100,13 @@ struct PairScheduler {
                     const int r0 = tc.mb * kPairBM;
                     const int g0 = __ldg(p.m_indices + r0);
                     const int g1 = r0 + kBM < p.M ? __ldg(p.m_indices + r0 + kBM) : -1;
-                    if (report && !second && (g0 >= p.G || g1 >= p.G))
+                    // a half whose first row is out of range, or is padding
+                    // over rows that carry a group index, breaks the
+                    // alignment rule: its rows stay untouched, and it is
+                    // flagged (once, on the first pass, at column block 0)
+                    if (report && !second && tc.nb == 0 &&
+                        (g0 >= p.G || g1 >= p.G || (g0 < 0 && padding_block_has_rows(p.m_indices, r0)) ||
+                         (g1 < 0 && r0 + kBM < p.M && padding_block_has_rows(p.m_indices, r0 + kBM))))
                         record_status(kCodeBadGroup, kRoleSched, 0);
                     const bool v0 = g0 >= 0 && g0 < p.G;
                     const bool v1 = g1 >= 0 && g1 < p.G;
@@ -126,13 +132,15 @@ struct PairScheduler {
 };
 
 // NWG promotion warpgroups split the tile's columns (BN / NWG each).  With
-// three, every promotion thread holds 64 columns and loads its whole partial
-// from TMEM in one round, so each buffer goes back to the MMA early; the
-// block is then 16 warps (three promotion warpgroups and one control
-// warpgroup: the two producers, the MMA warp and one idle warp), launched at
-// 128 registers a thread and rebalanced with setmaxnreg: 152 for each
-// promotion thread, 56 for the control warpgroup.
-template <int BN_, int STAGES_, int KS_, int NWG_ = 2>
+// REBAL (always for three or more warpgroups), the block gains an idle
+// fourth control warp, so that the two producers, the MMA warp and it form
+// one control warpgroup, and registers are rebalanced with setmaxnreg: the
+// block is launched at LAUNCH_REGS a thread, the control warpgroup drops to
+// CTRL_REGS and the promotion warpgroups take what is left (PROMO_REGS).
+// That lets each promotion thread hold its whole partial beside its
+// accumulator and load it from TMEM in one round (RMAX = BN_WG), so each
+// buffer goes back to the MMA after a single TMEM-load latency.
+template <int BN_, int STAGES_, int KS_, int NWG_ = 2, bool REBAL_ = false>
 struct PairConfig {
     static constexpr int BN = BN_;          // columns of the pair tile
     static constexpr int BN_HALF = BN / 2;  // B rows held by each CTA
@@ -140,19 +148,21 @@ struct PairConfig {
     static constexpr int KS = KS_;
     static constexpr int NUM_WG = NWG_;     // promotion warpgroups
     static constexpr int BN_WG = BN / NUM_WG;
+    static constexpr bool REBALANCE = REBAL_ || NUM_WG >= 3;
     // TMEM load rounds: the whole partial when it fits beside the
     // accumulator, else halves of up to 40 columns, else rounds of 32.
-    static constexpr int RMAX = BN_WG <= 64 ? BN_WG : (BN_WG <= 80 ? BN_WG / 2 : 32);
+    static constexpr int RMAX =
+        (BN_WG <= 64 || (REBALANCE && BN_WG <= 80)) ? BN_WG : (BN_WG <= 80 ? BN_WG / 2 : 32);
     static constexpr int NUM_PROMO_WARPS = 4 * NUM_WG;
     static constexpr int PRODUCER_A_WARP = NUM_PROMO_WARPS;
     static constexpr int PRODUCER_B_WARP = NUM_PROMO_WARPS + 1;
     static constexpr int MMA_WARP = NUM_PROMO_WARPS + 2;
-    static constexpr bool REBALANCE = NUM_WG == 3;
     static constexpr int CTRL_WARPS = REBALANCE ? 4 : 3;
     static constexpr int THREADS = (NUM_PROMO_WARPS + CTRL_WARPS) * 32;
-    static constexpr int LAUNCH_REGS = REBALANCE ? 65536 / THREADS : 0;
-    static constexpr int PROMO_REGS = 152;
+    static constexpr int LAUNCH_REGS = REBALANCE ? (65536 / THREADS) / 8 * 8 : 0;
     static constexpr int CTRL_REGS = 56;
+    static constexpr int PROMO_REGS_FIT = REBALANCE ? (LAUNCH_REGS * THREADS - 128 * CTRL_REGS) / (NUM_WG * 128) / 8 * 8 : 0;
+    static constexpr int PROMO_REGS = PROMO_REGS_FIT > 256 ? 256 : PROMO_REGS_FIT;
     // Warpgroup columns start at multiples of BN_WG; when BN_WG divides 128
     // they never straddle a 128-wide weight block, so one scale serves them.
     static constexpr bool UNIFORM_SCALE = (128 % (BN / NWG_) == 0) && (BN % (BN / NWG_) == 0);
@@ -167,7 +177,8 @@ struct PairConfig {
     // full, sfull, empty, sread per stage; tfull, tempty per TMEM buffer
     static constexpr int BAR_BYTES = 8 * (4 * STAGES + 2 * NBUF) + 16;
     // Epilogue boxes of 32 columns (64-byte rows, 64-byte swizzle), one
-    // staging buffer per warpgroup, plus one 16-column remainder box.
+    // staging buffer per warpgroup, plus one remainder box of the leftover
+    // columns (a multiple of 8).
     static constexpr int EPI_BOX = 32;
     static constexpr int EPI_FULL_BOXES = BN_WG / EPI_BOX;
     static constexpr int EPI_REM = BN_WG % EPI_BOX;
@@ -182,15 +193,15 @@ struct PairConfig {
     static constexpr int SMEM_BYTES = 1024 /*align slack*/ + EPI_OFFSET + NUM_WG * EPI_BUFS * EPI_WG_BYTES;
 
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair MMA N (M = 256): multiple of 32 up to 256");
-    static_assert(BN % NUM_WG == 0 && (NUM_WG == 2 || NUM_WG == 3), "promotion warpgroups");
+    static_assert(BN % NUM_WG == 0 && NUM_WG >= 2 && NUM_WG <= 4, "promotion warpgroups");
     static_assert(!REBALANCE || (NUM_WG * 128 * PROMO_REGS + 128 * CTRL_REGS <= THREADS * LAUNCH_REGS &&
-                                 LAUNCH_REGS % 8 == 0),
+                                 LAUNCH_REGS % 8 == 0 && PROMO_REGS >= LAUNCH_REGS && CTRL_REGS <= LAUNCH_REGS),
                   "setmaxnreg budgets must fit the registers the block is launched with");
-    static_assert(BN_WG % 16 == 0 && BN_WG <= 128, "promotion columns per warpgroup");
+    static_assert(BN_WG % 8 == 0 && BN_WG <= 128, "promotion columns per warpgroup");
     static_assert(B_BYTES % 1024 == 0, "B tiles must keep 1024-byte swizzle atoms aligned");
     static_assert(NBUF >= 2, "double-buffered TMEM at least");
     static_assert(KS >= 1 && KS <= 4, "K blocks per stage");
-    static_assert(EPI_REM == 0 || EPI_REM == 16, "remainder box of 16 columns");
+    static_assert(EPI_REM % 8 == 0, "remainder box of whole 16-byte rows");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -209,14 +220,14 @@ __device__ __forceinline__ bool pair_warp_wait(uint32_t bar, uint32_t parity, ui
     return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
-template <int BN, int STAGES, int KS, int LAYOUT, int NWG>
-__global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG>::THREADS, 1)
+template <int BN, int STAGES, int KS, int LAYOUT, int NWG, bool REBAL = false>
+__global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG, REBAL>::THREADS, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                          const __grid_constant__ CUtensorMap tmap_b,
                          const __grid_constant__ CUtensorMap tmap_dbox,
                          const __grid_constant__ CUtensorMap tmap_drem, const GemmParams p)
 {
-    using Cfg = PairConfig<BN, STAGES, KS, NWG>;
+    using Cfg = PairConfig<BN, STAGES, KS, NWG, REBAL>;
     constexpr int BN_WG = Cfg::BN_WG;
     constexpr int RMAX = Cfg::RMAX;
     constexpr int NBUF = Cfg::NBUF;
@@ -243,6 +254,7 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG>::THREADS, 1)
     const int lane = threadIdx.x % 32;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
+    stamp_start(p);
 
     if (warp == Cfg::PRODUCER_A_WARP && lane == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -454,10 +466,13 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG>::THREADS, 1)
                 row_ok = m_local < p.M;
             } else if constexpr (LAYOUT == kContiguous) {
                 row_ok = false;
+                // a row is computed when its index is this visit's group and
+                // the group of its own 128-row block (the group of the
+                // block's first row)
                 const int block_g = m_half < p.M ? __ldg(p.m_indices + m_half) : -1;
                 if (m_local < p.M && block_g >= 0) {
                     const int idx = __ldg(p.m_indices + m_local);
-                    row_ok = idx == tc.g;
+                    row_ok = idx == tc.g && idx == block_g;
                     if (idx >= 0 && idx != block_g)
                         record_status(kCodeBadGroup, kRolePromote, 1);
                 }
@@ -620,6 +635,7 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG>::THREADS, 1)
     // no CTA leaves (or frees TMEM) while its peer may still signal its
     // barriers or the leader's MMAs may still write its TMEM
     cluster_sync();
+    stamp_end(p);
     if (warp == Cfg::MMA_WARP) {
         tc_fence_after_sync();
         tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);

@@ -496,6 +496,13 @@ __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld_32x32b_x4(uint32_t taddr, uint32_t (&r)[4])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+}
+
 // 32 lanes x 4 consecutive 32-bit columns: thread i of the warp writes v to
 // lane (taddr.lane + i), columns taddr.col .. taddr.col+3.  Whole warp.
 __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v)
