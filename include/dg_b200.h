@@ -206,20 +206,23 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA,
 
 /*
  * Dense NT GEMM that allocates no device memory (same arguments, layouts
- * and result as dg_fp8_gemm_nt).  The pages describe no such call; it exists
- * for callers that cannot call cudaMalloc while they run: code being
- * captured into a CUDA graph (allocation is not allowed during capture),
- * code whose framework owns all device memory through its own caching pool,
- * and latency-critical loops where the device-wide synchronisation that
- * cudaMalloc/cudaFree may imply is not acceptable.
+ * and result as dg_fp8_gemm_nt).  The pages describe no such call.  It is
+ * for callers that cannot let a library allocate device memory while they
+ * run: frameworks that hand out all device memory from their own caching
+ * pool (an outside cudaMalloc can fail once the pool holds the memory, or
+ * fragment it), and latency-critical loops where the device-wide
+ * synchronisation that cudaMalloc/cudaFree may cause is not acceptable.
  *
  * It runs the K-split kernel (128 x 144 tiles, each tile's K range split
- * over a cluster of S = 1..16 CTAs) with the fp32 partials in a fixed
- * 32 MiB array compiled into the library, which every GPU that loads the
- * library holds until the process exits.  The partials of one call take
- * ceil(M/128) * ceil(N/144) * S * 73,728 bytes; S is lowered until they fit,
- * and a problem that does not fit even with S = 1 is rejected with
- * DG_ERR_WORKSPACE_LIMIT before anything is launched.
+ * over a cluster of S CTAs) with the fp32 partials in a fixed 32 MiB array
+ * compiled into the library, which every GPU that loads the library holds
+ * until the process exits.  S is the dense planner's split for the shape
+ * when it splits, else the largest of 16, 8, 4, 2 that gives every split the
+ * same number (at least two) of K blocks and whose cluster fits the SM cap
+ * (dg_set_num_sms); it is lowered (by the same rule, down to 1) until the
+ * partials, ceil(M/128) * ceil(N/144) * S * 73,728 bytes, fit.  A problem
+ * that does not fit even with S = 1 is rejected with DG_ERR_WORKSPACE_LIMIT
+ * before anything is launched.  dg_describe_config layout 6 reports S.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
@@ -228,6 +231,7 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA,
  *    overlap on the GPU (different streams, or a graph that runs them
  *    concurrently) race on the array: serialise them.
  *  - No cudaMalloc, cudaFree or other allocating routine is called.
+ *  - If dg_get_device_status reports DG_ERR_TIMEOUT, D is undefined.
  */
 dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, const void *B,
                                    const float *sB, void *D, int M, int N, int K,
@@ -328,10 +332,37 @@ int dg_get_num_sms(void);
 #define DG_TILES_PAIR 2
 dg_status_t dg_set_tile_family(int family);
 
+/* Pins the planner's tile width (BLOCK_N) to n, one of the compiled widths
+ * (112, 128, 144, 160, 192, 224, 256; 144 is the K-split decode tile), or 0
+ * to let the cost model decide (the default; DG_FORCE_BLOCK_N sets the
+ * initial value).  Process-wide, for tuning and tests: a call whose layout
+ * and tile family have no tile of that width takes the first tile of its
+ * table.  Returns DG_ERR_INVALID_ARG for any other n.  (A tuning control of
+ * this library; the pages have no counterpart.) */
+dg_status_t dg_set_block_n(int n);
+
+/* Launch timing.  While `stamps` (a DEVICE array of two unsigned 64-bit
+ * integers, 8-byte aligned) is set, every GEMM launch folds the %globaltimer
+ * time (ns) at which its first CTA started into stamps[0] (atomic minimum)
+ * and the time at which its last CTA ended into stamps[1] (atomic maximum):
+ * the caller sets stamps[0] = UINT64_MAX and stamps[1] = 0 before the
+ * launches it wants to span, and stamps[1] - stamps[0] is their duration on
+ * the device, without launch latency.  NULL (the default) turns it off.
+ * Process-wide; the cost is two atomics per CTA.  (A measurement hook of
+ * this library; the pages have no counterpart.) */
+dg_status_t dg_set_timing_stamps(unsigned long long *stamps);
+
+/* Tensor maps (TMA descriptors) the library has encoded so far in this
+ * process.  Each call looks its maps up in a cache keyed by buffer address,
+ * shape, strides, box and swizzle, so a call repeated on the same buffers
+ * encodes none and leaves this count unchanged. */
+unsigned long long dg_get_tensor_map_encodes(void);
+
 /* Time limit of each pipeline wait inside the kernels, in nanoseconds
  * (default 2e9).  A wait that runs past it makes the kernel record
- * DG_ERR_TIMEOUT, drain its in-flight copies and return.  0 restores the
- * default. */
+ * DG_ERR_TIMEOUT, drain its in-flight copies and return.  The output of a
+ * call that reported DG_ERR_TIMEOUT is undefined (the K-split paths write NaN
+ * into the columns of a split that gave up).  0 restores the default. */
 dg_status_t dg_set_wait_timeout_ns(uint64_t ns);
 
 /* Test hook for the bounded-wait path (0 = off, the default).  While on,
@@ -354,9 +385,11 @@ dg_status_t dg_get_device_status_detail(cudaStream_t stream, uint32_t *word);
 
 /* Describes the kernel configuration the library would launch for a problem
  * (layout 0 = dense, 1 = contiguous, 2 = masked, and 3, 4, 5 for the same
- * layouts in the UE8M0 block-scaled mode; for masked, M = expected_m and
- * groups = G) into buf (NUL-terminated, truncated to len).  Returns the
- * number of characters it wanted to write, or -1 on bad arguments. */
+ * layouts in the UE8M0 block-scaled mode; 6 = dense through
+ * dg_fp8_gemm_nt_noalloc, ksplit=0 when it does not fit its scratch; for
+ * masked, M = expected_m and groups = G) into buf (NUL-terminated, truncated
+ * to len).  Returns the number of characters it wanted to write, or -1 on
+ * bad arguments. */
 int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf,
                        int len);
 

@@ -62,6 +62,9 @@ _SIGNATURES = {
     "dg_set_num_sms": (_I, [_I]),
     "dg_get_num_sms": (_I, []),
     "dg_set_tile_family": (_I, [_I]),
+    "dg_set_block_n": (_I, [_I]),
+    "dg_set_timing_stamps": (_I, [_P]),
+    "dg_get_tensor_map_encodes": (ctypes.c_ulonglong, []),
     "dg_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
     "dg_set_stall_injection": (_I, [_I]),
     "dg_get_device_status": (_I, [_P]),
@@ -158,6 +161,28 @@ DG_TILES_AUTO, DG_TILES_ONE_CTA, DG_TILES_PAIR = 0, 1, 2
 def dg_set_tile_family(family: int) -> None:
     """Restrict the planner to one tile family (DG_TILES_*); 0 = automatic."""
     _check("dg_set_tile_family", load_library().dg_set_tile_family(family))
+
+
+def dg_set_block_n(n: int) -> None:
+    """Pin the planner's tile width to a compiled BLOCK_N; 0 = automatic."""
+    _check("dg_set_block_n", load_library().dg_set_block_n(n))
+
+
+def dg_set_timing_stamps(stamps) -> None:
+    """Record each launch's first-CTA start / last-CTA end (%globaltimer ns)
+    into a CUDA int64 tensor of 2 elements (None turns it off)."""
+    if stamps is None:
+        _check("dg_set_timing_stamps", load_library().dg_set_timing_stamps(None))
+        return
+    ptr = _dev(stamps, "stamps", (torch.int64,), 1)
+    if stamps.numel() != 2:
+        raise ValueError("stamps must hold 2 elements")
+    _check("dg_set_timing_stamps", load_library().dg_set_timing_stamps(ptr))
+
+
+def dg_get_tensor_map_encodes() -> int:
+    """Tensor maps encoded so far (cache misses of the library's map cache)."""
+    return int(load_library().dg_get_tensor_map_encodes())
 
 
 def dg_set_wait_timeout_ns(ns: int) -> None:

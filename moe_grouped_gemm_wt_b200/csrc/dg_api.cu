@@ -29,6 +29,7 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 std::atomic<int> g_num_sms_cap{0};
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
 std::atomic<int> g_stall_injection{0};
+std::atomic<unsigned long long *> g_stamps{nullptr};  // dg_set_timing_stamps
 int g_sm_count[kMaxDevices] = {0};
 
 // ------------------------------------------------------------ driver entry
@@ -53,6 +54,79 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+// Tensor maps are cached per (base pointer, data type, shape, strides, box,
+// swizzle, L2 promotion): a call repeated on the same buffers encodes none,
+// which keeps the host cost of small, frequent calls (decode steps) down.
+// The cache is a small set-associative
+// table under a mutex; a miss encodes with cuTensorMapEncodeTiled and
+// replaces the set's entries in turn.  The device a map is used on does not
+// enter the key: the encoded map holds only the address and the layout.
+struct TmapKey {
+    const void *base;
+    uint64_t dims[3];
+    uint64_t strides[2];
+    uint32_t box[3];
+    uint32_t rank, dtype, swizzle, promo;
+    bool operator==(const TmapKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
+};
+
+constexpr int kTmapSets = 64;
+constexpr int kTmapWays = 4;
+struct TmapEntry {
+    bool valid = false;
+    TmapKey key;
+    CUtensorMap map;
+};
+std::mutex g_tmap_mutex;
+TmapEntry g_tmap_cache[kTmapSets][kTmapWays];
+int g_tmap_next_way[kTmapSets] = {};
+std::atomic<uint64_t> g_tmap_encodes{0};  // encodes performed (cache misses)
+
+bool encode_cached(CUtensorMap *map, CUtensorMapDataType dtype, uint32_t rank, const void *base,
+                   const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box,
+                   CUtensorMapSwizzle swizzle, CUtensorMapL2promotion promo)
+{
+    TmapKey k;
+    std::memset(&k, 0, sizeof(k));  // padding bytes take part in the comparison
+    k.base = base;
+    for (uint32_t i = 0; i < rank; ++i) {
+        k.dims[i] = dims[i];
+        k.box[i] = box[i];
+        if (i + 1 < rank)
+            k.strides[i] = strides[i];
+    }
+    k.rank = rank;
+    k.dtype = static_cast<uint32_t>(dtype);
+    k.swizzle = static_cast<uint32_t>(swizzle);
+    k.promo = static_cast<uint32_t>(promo);
+    uint64_t h = reinterpret_cast<uintptr_t>(base) >> 4;
+    for (uint32_t i = 0; i < rank; ++i)
+        h = h * 1000003u ^ (k.dims[i] * 31u + k.box[i]);
+    h = h * 1000003u ^ (k.dtype * 7u + k.swizzle * 3u + k.promo);
+    const int set = static_cast<int>((h ^ (h >> 29)) % kTmapSets);
+    std::lock_guard<std::mutex> lock(g_tmap_mutex);
+    for (TmapEntry &e : g_tmap_cache[set]) {
+        if (e.valid && e.key == k) {
+            *map = e.map;
+            return true;
+        }
+    }
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(map, dtype, rank, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    g_tmap_encodes.fetch_add(1);
+    TmapEntry &slot = g_tmap_cache[set][g_tmap_next_way[set]];
+    g_tmap_next_way[set] = (g_tmap_next_way[set] + 1) % kTmapWays;
+    slot.valid = true;
+    slot.key = k;
+    slot.map = *map;
+    return true;
+}
+
 // An e4m3 operand [rows][K] viewed in 3-D as (byte within a 128-wide K
 // block, row, K block), so that one box of [ks][box_rows][128 bytes] fetches
 // ks consecutive K blocks of box_rows rows, each block a 128-byte-swizzled
@@ -60,49 +134,33 @@ EncodeTiledFn encode_fn()
 bool make_tmap_operand(CUtensorMap *map, const void *base, uint64_t K, uint64_t rows,
                        uint32_t box_rows, uint32_t ks)
 {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc)
-        return false;
     cuuint64_t dims[3] = {128, rows, K / 128};
     cuuint64_t strides[2] = {K, 128};
     cuuint32_t box[3] = {128, box_rows, ks};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 // An MN-major e4m3 operand stored [K][inner] (inner = M for A, N for B):
 // 2-D boxes of 128 inner bytes by box_k K rows, 128-byte swizzled.
 bool make_tmap_mn(CUtensorMap *map, const void *base, uint64_t inner, uint64_t K, uint32_t box_k)
 {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc)
-        return false;
     cuuint64_t dims[2] = {inner, K};
     cuuint64_t strides[1] = {inner};
     cuuint32_t box[2] = {128, box_k};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 // 2-D bf16 matrix [rows][inner] (the output), box [box_rows][box_inner].
 bool make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                     uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle)
 {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc)
-        return false;
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {inner * 2};
     cuuint32_t box[2] = {box_inner, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, swizzle,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE);
 }
 
 // ------------------------------------------------------------------- device
@@ -179,23 +237,27 @@ struct TileChoice {
     double kb_ns;    // measured time of one K block of one tile (cost model, us)
     int pair;        // 1: 256 x bn tiles on CTA pairs (cta_group::2)
     double tile_us;  // per-tile fill, drain and epilogue (cost model, us)
-    int wg = 2;      // promotion warpgroups (pair tiles: 2 or 3)
+    int wg = 2;      // promotion warpgroups
+    int rebal = 0;   // pair tiles: registers rebalanced with setmaxnreg (always for wg >= 3)
 };
 constexpr TileChoice kTileChoices[] = {
     {112, 3, 2, 0, 0.41, 0, 1.9}, {128, 5, 1, 0, 0.53, 0, 1.9}, {224, 2, 2, 0, 0.78, 0, 1.9},
-    {256, 3, 1, 0, 0.68, 0, 1.9}, {144, 3, 2, 1, 0.40, 0, 1.9}, {160, 3, 2, 0, 0.441, 1, 2.2},
+    {256, 3, 1, 0, 0.68, 0, 1.9}, {144, 3, 2, 1, 0.40, 0, 1.9, 3}, {160, 3, 2, 0, 0.441, 1, 2.2},
     {192, 3, 2, 0, 0.50, 1, 2.2, 3},
 };
 constexpr int kSplitFixedNs = 1500;  // cluster reduction + pipeline fill of a split CTA
 
-// DG_FORCE_BLOCK_N=<n> pins the tile width to one of the compiled choices
-// (read once; for tuning sweeps).
+// Tile width pinned by dg_set_block_n (0 = the cost model decides); its
+// initial value comes from DG_FORCE_BLOCK_N=<n>.
+std::atomic<int> g_forced_bn{-1};
+
 int forced_block_n()
 {
-    static int v = -1;
+    int v = g_forced_bn.load();
     if (v < 0) {
         const char *e = std::getenv("DG_FORCE_BLOCK_N");
-        v = e ? std::atoi(e) : 0;
+        g_forced_bn.compare_exchange_strong(v, e ? std::atoi(e) : 0);
+        v = g_forced_bn.load();
     }
     return v;
 }
@@ -328,11 +390,11 @@ int choose_raster(int num_mb)
     return num_mb < want ? (num_mb > 0 ? num_mb : 1) : want;
 }
 
-template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false>
+template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false, int NWG = 2>
 dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
                           const GemmParams &p, int grid, cudaStream_t stream)
 {
-    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == dg::kKGrouped>;
+    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == dg::kKGrouped, NWG>;
     CUtensorMap ta, tb;
     const bool ok_a = A_MN ? make_tmap_mn(&ta, A, a_rows, static_cast<uint64_t>(p.K), KS * dg::kBK)
                            : make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS);
@@ -354,7 +416,7 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
     } else {
         tdrem = td64;
     }
-    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT, SPLIT, A_MN, B_MN>;
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT, SPLIT, A_MN, B_MN, NWG>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices)
@@ -397,17 +459,17 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
 
 // Pair tiles: a cluster of two CTAs per 256 x BN tile, persistent over
 // tiles; grid = 2 x (pairs in use).
-template <int BN, int STAGES, int KS, int LAYOUT, int NWG>
+template <int BN, int STAGES, int KS, int LAYOUT, int NWG, bool REBAL = false>
 dg_status_t launch_pair(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
                         const GemmParams &p, int grid, cudaStream_t stream)
 {
-    using Cfg = PairConfig<BN, STAGES, KS, NWG>;
+    using Cfg = PairConfig<BN, STAGES, KS, NWG, REBAL>;
     CUtensorMap ta, tb;
     if (!make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS) ||
         !make_tmap_operand(&tb, B, static_cast<uint64_t>(p.K), b_rows, Cfg::BN_HALF, KS))
         return DG_ERR_CUDA;
     // output boxes of 128 rows: 32 columns with 64-byte swizzle, and a
-    // 16-column unswizzled remainder box
+    // unswizzled remainder box of the leftover columns
     CUtensorMap tdbox, tdrem;
     if (!make_tmap_bf16(&tdbox, p.D, static_cast<uint64_t>(p.N), a_rows, Cfg::EPI_BOX, dg::kBM,
                         CU_TENSOR_MAP_SWIZZLE_64B))
@@ -419,7 +481,7 @@ dg_status_t launch_pair(const void *A, uint64_t a_rows, const void *B, uint64_t 
     } else {
         tdrem = tdbox;
     }
-    auto kern = dg::fp8_gemm_pair_kernel<BN, STAGES, KS, LAYOUT, NWG>;
+    auto kern = dg::fp8_gemm_pair_kernel<BN, STAGES, KS, LAYOUT, NWG, REBAL>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices)
@@ -472,11 +534,11 @@ dg_status_t launch_pair(const void *A, uint64_t a_rows, const void *B, uint64_t 
 // Co-resident clusters of S CTAs of a split configuration (cached per
 // device).  The split kernel keeps one tile per cluster, so a plan is only
 // used when every cluster of the grid fits at once.
-template <int BN, int STAGES, int KS>
+template <int BN, int STAGES, int KS, int NWG>
 int query_max_clusters(int S)
 {
-    using Cfg = KernelConfig<BN, STAGES, KS, true>;
-    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, dg::kDense, true>;
+    using Cfg = KernelConfig<BN, STAGES, KS, true, false, NWG>;
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, dg::kDense, true, false, false, NWG>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) !=
             cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
@@ -505,14 +567,19 @@ int query_max_clusters(int S)
 int max_active_clusters(const TileChoice &c, int S)
 {
     static int cache[kMaxDevices][5] = {};  // S = 2, 4, 8, 16 (index log2(S))
-    const int dev = current_device();
-    if (dev < 0 || dev >= kMaxDevices || c.bn != 144)
+    if (c.bn != 144 || S < 1)
         return 0;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) {
+        // no device (host-only planning, dg_describe_config): one CTA per SM
+        const int cap = g_num_sms_cap.load();
+        return (cap > 0 ? cap : 148) / S;
+    }
     int idx = 0;
     while ((2 << idx) < S)
         ++idx;
     if (cache[dev][idx] == 0) {
-        const int n = query_max_clusters<144, 3, 2>(S);
+        const int n = query_max_clusters<144, 3, 2, 3>(S);
         cache[dev][idx] = n > 0 ? n : -1;
     }
     // The SM cap (dg_set_num_sms) bounds the clusters too.
@@ -543,8 +610,12 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
             grid_pairs = static_cast<int>(ptiles);
         if (grid_pairs <= 0)
             return DG_OK;
-        if (c.bn == 160 && c.stages == 3 && c.ks == 2 && c.wg == 2)
+        if (c.bn == 160 && c.stages == 3 && c.ks == 2 && c.wg == 2 && !c.rebal)
             return launch_pair<160, 3, 2, LAYOUT, 2>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
+        if (c.bn == 160 && c.stages == 3 && c.ks == 2 && c.wg == 2 && c.rebal)
+            return launch_pair<160, 3, 2, LAYOUT, 2, true>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
+        if (c.bn == 160 && c.stages == 3 && c.ks == 2 && c.wg == 4)
+            return launch_pair<160, 3, 2, LAYOUT, 4>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
         if (c.bn == 192 && c.stages == 3 && c.ks == 2 && c.wg == 3)
             return launch_pair<192, 3, 2, LAYOUT, 3>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
         return DG_ERR_UNSUPPORTED;
@@ -579,9 +650,9 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
     DG_TILE_CASE(256, 3, 1)
 #undef DG_TILE_CASE
     if constexpr (LAYOUT == dg::kDense && !B_MN) {
-        if (c.bn == 144 && c.stages == 3 && c.ks == 2 && c.split)
-            return launch_kernel<144, 3, 2, LAYOUT, true, A_MN, false>(A, a_rows, B, b_rows, p, grid,
-                                                                       stream);
+        if (c.bn == 144 && c.stages == 3 && c.ks == 2 && c.split && c.wg == 3)
+            return launch_kernel<144, 3, 2, LAYOUT, true, A_MN, false, 3>(A, a_rows, B, b_rows, p, grid,
+                                                                          stream);
     }
     return DG_ERR_UNSUPPORTED;
 }
@@ -633,6 +704,7 @@ dg_status_t dense_gemm(const void *A, const float *sA, const void *B, const floa
     p.num_mb = (M + 127) / 128;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
+    p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
     const int limits = (a_mn || b_mn ? kNoPair : 0) | (b_mn ? kWholeBoxes : 0);
     const Plan plan = choose_plan(p.num_mb, (M + 255) / 256, N, p.num_kb, sms, true, limits);
@@ -918,9 +990,16 @@ GemmParams bs_params(const int32_t *sfa, const int32_t *sfb, void *D, int M, int
     p.num_mb = (M + 127) / 128;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
+    p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
     return p;
 }
+
+// Fixed scratch of dg_fp8_gemm_nt_noalloc and the tile width of the K-split
+// kernel it runs.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+constexpr int kNoAllocBN = 144;
+int noalloc_split(int M, int N, int K, int sms);
 
 }  // namespace
 
@@ -996,6 +1075,7 @@ dg_status_t dg_fp8_k_grouped_gemm_tn_contiguous(const void *A, const float *sA, 
     p.num_mb = (M + 127) / 128;
     p.raster = 1;
     p.timeout_ns = g_timeout_ns.load();
+    p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
     const int avg_kb = p.num_kb / num_groups > 0 ? p.num_kb / num_groups : 1;
     const Plan plan = choose_plan(static_cast<int64_t>(num_groups) * p.num_mb, 0, N, avg_kb, sms, false,
@@ -1041,6 +1121,7 @@ dg_status_t dg_fp8_gemm_nt_acc(const void *A, const float *sA, const void *B, co
     p.num_mb = (M + 127) / 128;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
+    p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
     const Plan plan = choose_plan(p.num_mb, (M + 255) / 256, N, p.num_kb, sms, true);
     if (print_configs())
@@ -1087,6 +1168,7 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const
     p.num_mb = M_total / 128;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
+    p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
     const Plan plan = choose_plan(p.num_mb, (M_total + 255) / 256, N, p.num_kb, sms, false);
     if (print_configs())
@@ -1133,6 +1215,7 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const voi
     p.num_mb = (max_m + 127) / 128;
     p.raster = 1;
     p.timeout_ns = g_timeout_ns.load();
+    p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
     const int em = (expected_m > 0 && expected_m < max_m) ? expected_m : max_m;
     const Plan plan = choose_plan(static_cast<int64_t>(num_groups) * ((em + 127) / 128),
@@ -1288,6 +1371,29 @@ dg_status_t dg_set_tile_family(int family)
     return DG_OK;
 }
 
+dg_status_t dg_set_block_n(int n)
+{
+    bool known = n == 0;
+    for (const TileChoice &c : kTileChoices)
+        known = known || c.bn == n;
+    for (const BsChoice &c : kBsChoices)
+        known = known || c.bn == n;
+    if (!known)
+        return DG_ERR_INVALID_ARG;
+    g_forced_bn.store(n);
+    return DG_OK;
+}
+
+unsigned long long dg_get_tensor_map_encodes(void) { return g_tmap_encodes.load(); }
+
+dg_status_t dg_set_timing_stamps(unsigned long long *stamps)
+{
+    if (stamps != nullptr && !aligned(stamps, 8))
+        return DG_ERR_ALIGNMENT;
+    g_stamps.store(stamps);
+    return DG_OK;
+}
+
 dg_status_t dg_set_wait_timeout_ns(uint64_t ns)
 {
     g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
@@ -1329,13 +1435,21 @@ dg_status_t dg_get_device_status(cudaStream_t stream)
 
 int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, int len)
 {
-    if (layout < 0 || layout > 5 || M < 0 || N <= 0 || K <= 0 || groups <= 0 || (len > 0 && !buf))
+    if (layout < 0 || layout > 6 || M < 0 || N <= 0 || K <= 0 || groups <= 0 || (len > 0 && !buf))
         return -1;
     // Without a device (host-only use) the SM cap alone decides, else 148.
     const int dev = current_device();
     int sms = effective_sms(dev);
     if (sms <= 0)
         sms = g_num_sms_cap.load() > 0 ? g_num_sms_cap.load() : 148;
+    if (layout == 6) {
+        // the dense GEMM through dg_fp8_gemm_nt_noalloc (ksplit=0: too large
+        // for its fixed scratch)
+        return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
+                             "layout=6 BM=128 BN=%d BK=128 stages=3 ks=2 ksplit=%d pair=0 wg=2 sms=%d m_blocks=%d n_blocks=%d noalloc=1",
+                             kNoAllocBN, noalloc_split(M, N, K - K % 128, sms), sms, (M + 127) / 128,
+                             (N + kNoAllocBN - 1) / kNoAllocBN);
+    }
     if (layout >= 3) {
         // the UE8M0 block-scaled mode (one-CTA or pair tiles, no K split)
         const int64_t mb = static_cast<int64_t>((M + 127) / 128) * (layout == 5 ? groups : 1);
@@ -1384,17 +1498,41 @@ const char *dg_status_string(dg_status_t status)
 //
 // dg_fp8_gemm_nt_noalloc: the dense GEMM through the K-split kernel, with the
 // split partials in a fixed array compiled into this library instead of a
-// workspace obtained with cudaMalloc.  For callers that must not allocate
-// device memory while they run: code being captured into a CUDA graph
-// (allocation is not allowed during capture), code whose framework keeps
-// all device memory in its own caching pool (an allocation behind its back
-// can fail or fragment that pool), and latency-critical loops where the
-// device-wide synchronisation that cudaMalloc/cudaFree may imply is not
-// acceptable.
+// workspace obtained with cudaMalloc.  For callers that must not have device
+// memory allocated behind their back: frameworks whose caching pool hands
+// out all device memory (an outside allocation can fail or fragment that
+// pool), and latency-critical loops where the device-wide synchronisation
+// that cudaMalloc/cudaFree may cause is not acceptable.
 
 namespace {
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+
+// Split count of the no-allocation path for an M x N x K problem on `sms`
+// SMs: the planner's own when it splits this shape, else the largest of
+// 16, 8, 4, 2 that gives every split the same number (at least two) of K
+// blocks -- no split is left empty -- and whose cluster the device can
+// schedule within the SM cap; then lowered (through the same rule, down to
+// 1) until the partials fit the fixed scratch.  Returns 0 when even S = 1
+// does not fit.
+int noalloc_split(int M, int N, int K, int sms)
+{
+    const int num_kb = K / 128;
+    const int64_t tiles = static_cast<int64_t>((M + 127) / 128) * ((N + kNoAllocBN - 1) / kNoAllocBN);
+    const size_t per_split = static_cast<size_t>(tiles) * kNoAllocBN * dg::kBM * sizeof(float);
+    auto usable = [&](int S) {
+        if (S == 1)
+            return true;
+        const int kbps = (num_kb + S - 1) / S;
+        if (kbps < 2 || (num_kb + kbps - 1) / kbps != S || S > sms)
+            return false;
+        return max_active_clusters(kTileChoices[4], S) > 0;
+    };
+    const Plan plan = choose_plan((M + 127) / 128, (M + 255) / 256, N, num_kb, sms, true);
+    int S = (plan.c.split && plan.c.bn == kNoAllocBN) ? plan.ksplit : 16;
+    while (S > 1 && (!usable(S) || per_split * S > kNoAllocScratchBytes))
+        S /= 2;
+    return per_split * S > kNoAllocScratchBytes ? 0 : S;
 }
+}  // namespace
 
 // The fixed scratch.  Every GPU that loads this library holds it until the
 // process exits.  Host code must not use this name as a device address (on
@@ -1443,11 +1581,11 @@ extern "C" dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, co
     if (sms <= 0)
         return DG_ERR_CUDA;
 
-    // The K-split kernel's tile (BN = 144).  The split count is the one the
-    // planner would use for this shape when it splits, else the largest
-    // power of two up to 16 that leaves every split at least two K blocks;
-    // it is halved until the partials fit the fixed scratch.
-    constexpr int kBN = 144;
+    // The K-split kernel's tile (BN = 144), split S ways (noalloc_split).
+    constexpr int kBN = kNoAllocBN;
+    const int S = noalloc_split(M, N, K, sms);
+    if (S == 0)
+        return DG_ERR_WORKSPACE_LIMIT;
     GemmParams p{};
     p.sA = sA;
     p.sB = sB;
@@ -1463,24 +1601,10 @@ extern "C" dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, co
     p.num_nb = (N + kBN - 1) / kBN;
     p.raster = choose_raster(p.num_mb);
     p.timeout_ns = g_timeout_ns.load();
+    p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
     const int64_t tiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
-    const Plan plan = choose_plan(p.num_mb, (M + 255) / 256, N, p.num_kb, sms, true);
-    int S = 1;
-    if (plan.c.split && plan.c.bn == kBN) {
-        S = plan.ksplit;
-    } else {
-        for (int cand = 16; cand >= 2; cand /= 2)
-            if ((p.num_kb + cand - 1) / cand >= 2) {
-                S = cand;
-                break;
-            }
-    }
     const size_t per_split = static_cast<size_t>(tiles) * kBN * dg::kBM * sizeof(float);
-    while (S > 1 && per_split * S > kNoAllocScratchBytes)
-        S /= 2;
-    if (per_split * S > kNoAllocScratchBytes)
-        return DG_ERR_WORKSPACE_LIMIT;
     p.ksplit = S;
     p.kb_per_split = (p.num_kb + S - 1) / S;
     st = noalloc_scratch_address(&p.ws);
