@@ -146,7 +146,7 @@ def test_ue8m0_describe_config(lib):
     # decode shape: too few pair tiles to fill the pairs, one-CTA tiles
     lib.dg_describe_config(3, 128, 2112, 7168, 1, buf, 256)
     assert dict(kv.split("=") for kv in buf.value.decode().split())["pair"] == "0"
-    assert lib.dg_describe_config(6, 128, 256, 512, 1, buf, 256) == -1
+    assert lib.dg_describe_config(7, 128, 256, 512, 1, buf, 256) == -1
 
 
 def test_ue8m0_planner_under_an_sm_cap(lib):
@@ -167,6 +167,45 @@ def test_ue8m0_planner_under_an_sm_cap(lib):
         assert (d["BN"], d["pair"]) == ("224", "0"), d
     finally:
         lib.dg_set_tile_family(0)
+        lib.dg_set_num_sms(0)
+
+
+def test_noalloc_split_choice_under_an_sm_cap(lib):
+    """The split count of dg_fp8_gemm_nt_noalloc (host only, dg_describe_config
+    layout 6): every split gets the same number (at least two) of K blocks,
+    a cluster never has more CTAs than the SM cap allows, and the partials
+    fit the fixed 32 MiB scratch (ksplit=0: the problem is refused)."""
+    buf = ctypes.create_string_buffer(256)
+
+    def split(M, N, K):
+        assert lib.dg_describe_config(6, M, N, K, 1, buf, 256) > 0
+        d = dict(kv.split("=") for kv in buf.value.decode().split())
+        assert d["noalloc"] == "1" and d["BN"] == "144"
+        return int(d["ksplit"])
+
+    def even(S, K):
+        nkb = K // 128
+        kbps = -(-nkb // S)
+        return S == 1 or (kbps >= 2 and -(-nkb // kbps) == S)
+
+    try:
+        for cap in (0, 7, 3, 2):
+            assert lib.dg_set_num_sms(cap) == 0
+            for M, N, K in [(128, 2112, 7168), (300, 2112, 1152), (2048, 2112, 256), (64, 1024, 2048),
+                            (1024, 2112, 7168), (128, 256, 1152)]:
+                S = split(M, N, K)
+                tiles = -(-M // 128) * -(-N // 144)
+                assert S >= 1 and even(S, K), (cap, M, N, K, S)
+                assert cap == 0 or S <= cap, (cap, S)
+                assert tiles * S * 144 * 128 * 4 <= 32 << 20
+        # 9 K blocks never split 4 ways (3 + 3 + 3 + 0 would leave a split empty)
+        assert lib.dg_set_num_sms(0) == 0
+        assert split(4096, 2112, 1152) == 0          # 480 tiles: too large even unsplit
+        assert split(1024, 2112, 1152) == 2
+        assert split(128, 2112, 7168) == 8            # the dense planner's own split
+        assert lib.dg_set_num_sms(7) == 0
+        assert split(128, 2112, 7168) == 4
+    finally:
         lib.dg_set_num_sms(0)
 
 

@@ -258,6 +258,35 @@ def test_masked_moe_decode_ue8m0_sampled(dg, oracle_mod):
     assert_close(np.concatenate(gots), np.concatenate(refs), "ue8m0 masked MoE decode (sampled)")
 
 
+@pytest.mark.slow
+def test_contiguous_moe_ue8m0_sampled(dg, oracle_mod):
+    """The contiguous MoE benchmark workload (8 experts x 4096 rows, N=7168,
+    K=2048) in the launch configuration the benchmark times (the default
+    plan: 256 x 224 pair tiles), on 20,004 sampled outputs, corners
+    included; no output keeps the sentinel."""
+    p = gi.make_workload("contiguous_moe", ue8m0=True)
+    plan = _plan(dg, 4, p["M"], p["N"], p["K"], p["G"])
+    dev = torch.device("cuda")
+    A = torch.from_numpy(p["A"]).to(dev)
+    B = torch.from_numpy(p["B"]).to(dev)
+    sfa, sfb = _packed(dg, oracle_mod, p["sA"], p["sB"])
+    mi = torch.from_numpy(p["m_indices"]).to(dev)
+    D = torch.full((p["M"], p["N"]), SENTINEL, dtype=torch.int16, device=dev).view(torch.bfloat16)
+    dg.dg_fp8_grouped_gemm_contiguous_ue8m0(A, sfa, B, sfb, D, mi)
+    assert dg.dg_get_device_status() == 0
+    got = bits(D)
+    assert not np.any(got == SENTINEL), plan
+    rng = np.random.default_rng(5)
+    r = np.concatenate([rng.integers(0, p["M"], 20000), [0, 0, p["M"] - 1, p["M"] - 1]])
+    c = np.concatenate([rng.integers(0, p["N"], 20000), [0, p["N"] - 1, 0, p["N"] - 1]])
+    g = p["m_indices"][r]
+    ref = np.empty(r.size, np.uint16)
+    for gg in np.unique(g):
+        sel = g == gg
+        _, ref[sel] = oracle_mod.gemm_nt_sampled(p["A"], p["sA"], p["B"][gg], p["sB"][gg], r[sel], c[sel])
+    assert_close(got[r, c], ref, f"ue8m0 contiguous MoE (sampled), plan {plan}")
+
+
 # ---------------------------------------------------------------- packing
 
 def test_transform_flags_non_power_of_two(dg):

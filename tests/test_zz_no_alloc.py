@@ -1,15 +1,16 @@
 """The dense GEMM entry point that allocates no device memory.
 
-Some callers cannot let a library call cudaMalloc while they run: code being
-captured into a CUDA graph (allocation is not allowed during capture), code
-whose framework owns all device memory in its own caching pool, and
-latency-critical loops that cannot afford the synchronisation an allocation
-may bring.  dg_fp8_gemm_nt_noalloc serves them by keeping its K-split
-partials in a fixed array inside the library.  This file checks, through the
-C ABI, that it gives the same results as dg_fp8_gemm_nt (within the parity
-tolerance of the other tests) on two calls in a row -- the second call finds
-the first call's partials still in the shared array -- and that it frees or
-allocates nothing while it runs.
+Some callers cannot let a library allocate device memory behind their back:
+frameworks that hand out all device memory from their own caching pool (an
+outside cudaMalloc can fail once the pool has taken the memory, or fragment
+it), and latency-critical loops in which the device-wide synchronisation that
+cudaMalloc or cudaFree may cause is not acceptable.  dg_fp8_gemm_nt_noalloc
+serves them by keeping its K-split partials in a fixed array inside the
+library.  This file checks, through the C ABI, that its results match both
+the CPU oracle and dg_fp8_gemm_nt (within the parity tolerance of the other
+tests) on calls in a row -- each later call finds the previous call's
+partials still in the shared array -- and that, once its kernel is loaded,
+its calls change the device's free memory by nothing.
 
 It sits in a file pytest collects last, so a run that stops at the first
 failure has already run every other test; it also passes alone in a fresh
@@ -43,27 +44,35 @@ def dg():
 @pytest.mark.parametrize("M,N,K", [
     (128, 2112, 7168),   # the decode benchmark shape
     (64, 1024, 2048),
-    (300, 2112, 1152),   # three row blocks, 9 K blocks (uneven split)
+    (300, 2112, 1152),   # three row blocks, 9 K blocks (split 2 ways: 5 + 4)
+    (1024, 2112, 896),   # 120 tiles: the scratch bounds the split
 ])
-def test_noalloc_matches_default_entry_point_twice(dg, M, N, K):
+def test_noalloc_matches_oracle_and_default_entry_point(dg, oracle_mod, M, N, K):
     p = gi.dense_problem(M, N, K, seed_a=300 + M, seed_b=400 + N)
+    _, oracle_ref = oracle_mod.gemm_nt(p["A"], p["sA"], p["B"], p["sB"], want_f64=False)
     A, sA, B, sB, D_ref = dev_dense(p)
     dg.dg_fp8_gemm_nt(A, sA, B, sB, D_ref)
     assert dg.dg_get_device_status() == 0
     ref = bits(D_ref)
+    assert_close(ref, oracle_ref, f"dg_fp8_gemm_nt vs oracle, {M}x{N}x{K}")
 
-    outs = [torch.empty_like(D_ref) for _ in range(2)]
+    outs = [torch.empty_like(D_ref) for _ in range(3)]
+    # the first call looks up the scratch address and loads the kernel; the
+    # two calls after it must leave the device's free memory unchanged
+    dg.dg_fp8_gemm_nt_noalloc(A, sA, B, sB, outs[0])
     torch.cuda.synchronize()
     free_before, _ = torch.cuda.mem_get_info()
-    for out in outs:
+    for out in outs[1:]:
         dg.dg_fp8_gemm_nt_noalloc(A, sA, B, sB, out)
-    assert dg.dg_get_device_status() == 0
     torch.cuda.synchronize()
     free_after, _ = torch.cuda.mem_get_info()
+    assert dg.dg_get_device_status() == 0
     assert free_after == free_before, "the no-allocation entry point changed free device memory"
 
     for i, out in enumerate(outs):
-        assert_close(bits(out), ref, f"no-alloc call {i + 1} vs dg_fp8_gemm_nt, {M}x{N}x{K}")
+        got = bits(out)
+        assert_close(got, oracle_ref, f"no-alloc call {i + 1} vs oracle, {M}x{N}x{K}")
+        assert_close(got, ref, f"no-alloc call {i + 1} vs dg_fp8_gemm_nt, {M}x{N}x{K}")
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(dg):
