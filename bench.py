@@ -257,6 +257,7 @@ def shard_experts(p, rank, world):
     g0, g1 = rank * G // world, (rank + 1) * G // world
     q = dict(p)
     q["G"] = g1 - g0
+    q["group0"] = g0  # the shard's first expert in the whole problem
     q["B"], q["sB"] = p["B"][g0:g1], p["sB"][g0:g1]
     if p["kind"] == "masked":
         for k in ("A", "sA", "masked_m"):
@@ -271,6 +272,7 @@ def shard_experts(p, rank, world):
     q["A"], q["sA"] = p["A"][lo:hi], p["sA"][lo:hi]
     q["m_indices"] = np.where(mi[lo:hi] >= 0, mi[lo:hi] - g0, -1).astype(np.int32)
     q["M"] = hi - lo
+    q["row0"] = lo  # the shard's first row in the whole problem
     return q
 
 
@@ -297,8 +299,11 @@ def make_problem(name, ue8m0):
     return p
 
 
-def time_kernel(torch, dg, p, d, steps, warmup, flush):
-    """Per-launch CUDA-event times (ms) with an L2 flush before each launch."""
+def time_kernel(torch, dg, p, d, steps, warmup, flush, kernel_times=None):
+    """Per-launch CUDA-event times (ms) with an L2 flush before each launch.
+    With kernel_times (a list), each launch's device time from its first CTA's
+    start to its last CTA's end (the library's %globaltimer stamps, ms) is
+    appended to it: the launch without the launch latency the events see."""
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         flush.zero_()
@@ -306,16 +311,62 @@ def time_kernel(torch, dg, p, d, steps, warmup, flush):
     torch.cuda.synchronize()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    for i in range(steps):
-        flush.zero_()
-        starts[i].record(stream)
-        call(dg, p, d)
-        ends[i].record(stream)
+    stamps = torch.zeros((steps, 2), dtype=torch.int64, device=d["A"].device)
+    stamps[:, 0] = 2 ** 63 - 1
+    try:
+        for i in range(steps):
+            flush.zero_()
+            if kernel_times is not None:
+                dg.dg_set_timing_stamps(stamps[i])
+            starts[i].record(stream)
+            call(dg, p, d)
+            ends[i].record(stream)
+    finally:
+        dg.dg_set_timing_stamps(None)
     torch.cuda.synchronize()
     st = dg.dg_get_device_status()
     if st != 0:
         raise RuntimeError(f"device status {dg.dg_status_string(st)} during the benchmark")
+    if kernel_times is not None:
+        v = stamps.cpu().numpy()
+        kernel_times.extend(((v[:, 1] - v[:, 0]) * 1e-6).tolist())
     return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def launch_floor_ms(torch, steps, flush):
+    """An empty kernel timed like the GEMM (flush, then events around one
+    launch): the launch latency inside every event-timed figure."""
+    stream = torch.cuda.current_stream()
+    out = []
+    for i in range(steps + 3):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        torch.cuda._sleep(0)
+        e.record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            out.append(s.elapsed_time(e))
+    return statistics.median(out)
+
+
+def host_us_per_call(torch, dg, p, d, calls=1000):
+    """Host time of one call of the C ABI function (through ctypes, no
+    binding checks) over back-to-back enqueues: validation, planning, the
+    tensor-map cache lookup and the launch."""
+    lib = dg.load_library()
+    torch.cuda.synchronize()
+    if p["kind"] != "dense" or p.get("ue8m0"):
+        return None
+    args = [d["A"].data_ptr(), d["sA"].data_ptr(), d["B"].data_ptr(), d["sB"].data_ptr(), d["D"].data_ptr(),
+            p["M"], p["N"], p["K"], None]
+    lib.dg_fp8_gemm_nt(*args)
+    t0 = time.perf_counter()
+    for _ in range(calls):
+        lib.dg_fp8_gemm_nt(*args)
+    t1 = time.perf_counter()
+    torch.cuda.synchronize()
+    return (t1 - t0) / calls * 1e6
 
 
 def time_e2e(torch, dg, p, steps, warmup, dev):
@@ -445,9 +496,12 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    times = time_kernel(torch, dg, p, d, args.steps, max(args.warmup, 3), flush)
+    ktimes = []
+    times = time_kernel(torch, dg, p, d, args.steps, max(args.warmup, 3), flush, ktimes)
     torch.cuda.synchronize()
     ms = reduce_max_ms(sum(times) / len(times), dist, dev, world)
+    kernel_ms = reduce_max_ms(sum(ktimes) / len(ktimes), dist, dev, world)
+    floor_ms = launch_floor_ms(torch, 10, flush)
     if world > 1:
         dist.barrier()
 
@@ -460,14 +514,17 @@ def run_ours(args):
             same = name == args.workload and not expert_parallel and sweep_ue8m0 == ue8m0
             q = p if same else make_problem(name, sweep_ue8m0)
             dq = d if same else to_device(q, torch, dev, dg)
-            tq = time_kernel(torch, dg, q, dq, max(10, min(args.steps, 30)), 3, flush)
+            kq = []
+            tq = time_kernel(torch, dg, q, dq, max(10, min(args.steps, 30)), 3, flush, kq)
             mq = statistics.median(tq)
+            kmq = statistics.median(kq)
             fq, bq, rows = workload_cost(q)
             bound, t_roof, _ = roofline(fq, bq, pk)
             out[name] = {
                 "us": mq * 1e3, "tflops": fq / (mq * 1e-3) / 1e12,
                 "bound": bound, "roofline_us": t_roof * 1e6,
                 "frac_of_roofline": t_roof / (mq * 1e-3),
+                "kernel_us": kmq * 1e3, "kernel_frac_of_roofline": t_roof / (kmq * 1e-3),
                 "valid_rows": rows, "tile": tile_label(dg, q),
             }
             if not same:
@@ -483,6 +540,7 @@ def run_ours(args):
     clocks = sampler.stop()
 
     e2e_ms, h2d, d2h = time_e2e(torch, dg, p, max(10, min(args.steps, 50)), 3, dev)
+    host_us = host_us_per_call(torch, dg, p, d)
 
     value = flop_job / (ms * 1e-3) / 1e12 if expert_parallel else whole_job_value(flop, world, ms)
     bound, t_roof, fp8_peak = roofline(flop, byts, pk)
@@ -526,6 +584,13 @@ def run_ours(args):
                    "scales": "ue8m0 (separately declared block-scaled mode)" if ue8m0 else "fp32"},
         "roofline": roof,
         "frac_of_roofline": t_roof / (ms * 1e-3),
+        # the same launches timed on the device from the first CTA's start to
+        # the last CTA's end (%globaltimer stamps), and an empty kernel timed
+        # like the GEMM: the event-timed figure is roughly their sum
+        "kernel_us": kernel_ms * 1e3,
+        "kernel_frac_of_roofline": t_roof / (kernel_ms * 1e-3),
+        "launch_floor_us": floor_ms * 1e3,
+        "host_us_per_call": host_us,
         "cpu_baseline": cpu,
         "e2e": {"value": flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
