@@ -377,16 +377,24 @@ Plan choose_plan(int64_t m_blocks, int64_t pair_rows, int N, int num_kb, int sms
 }
 
 // Rasterisation: tiles are visited in groups of `raster` m-block rows (pair
-// rows for pair tiles), column by column inside a group.  DG_RASTER=<n>
-// overrides the group height (read once; for tuning sweeps).
-int choose_raster(int num_mb)
+// rows for pair tiles), column by column inside a group, so the CTAs working
+// at one time share the group's rows of A and walk B column by column.  The
+// group height is chosen so that the group's A rows (rows_per_block x K
+// bytes each) take at most about a third of L2 (40 MB): they then stay
+// resident while B streams past, and A is read from DRAM about once per
+// group instead of once per wave of tiles (at most 16 blocks per group).
+// DG_RASTER=<n> overrides the group height (read once; for tuning sweeps).
+int choose_raster(int num_mb, int rows_per_block, int K)
 {
     static int forced = -1;
     if (forced < 0) {
         const char *e = std::getenv("DG_RASTER");
         forced = e ? std::atoi(e) : 0;
     }
-    const int want = forced > 0 ? forced : 16;
+    constexpr double kBandBytes = 40.0 * 1024 * 1024;
+    const double block_bytes = static_cast<double>(rows_per_block) * (K > 0 ? K : 1);
+    int want = forced > 0 ? forced : static_cast<int>(kBandBytes / block_bytes);
+    want = want < 1 ? 1 : (want > 16 && forced <= 0 ? 16 : want);
     return num_mb < want ? (num_mb > 0 ? num_mb : 1) : want;
 }
 
@@ -431,8 +439,12 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
         attr_set[dev].store(true);
     }
     if (SPLIT) {
+        // 3-D grid: x the K split (a cluster along x), y the column tile, z
+        // the 128-row block -- one tile per cluster
+        (void)grid;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+        cfg.gridDim = dim3(static_cast<unsigned>(p.ksplit), static_cast<unsigned>(p.num_nb),
+                           static_cast<unsigned>(p.num_mb));
         cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
         cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
         cfg.stream = stream;
@@ -600,7 +612,7 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
         // the pair scheduler counts 256-row pair rows
         p.num_mb = (p.num_mb + 1) / 2;
         if (LAYOUT != dg::kMasked)
-            p.raster = choose_raster(p.num_mb);
+            p.raster = choose_raster(p.num_mb, 2 * dg::kBM, p.K);
         p.ksplit = 1;
         p.kb_per_split = p.num_kb;
         const int pairs = sms / 2;
@@ -616,6 +628,8 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
             return launch_pair<160, 3, 2, LAYOUT, 2, true>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
         if (c.bn == 160 && c.stages == 3 && c.ks == 2 && c.wg == 4)
             return launch_pair<160, 3, 2, LAYOUT, 4>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
+        if (c.bn == 128 && c.stages == 4 && c.ks == 2 && c.wg == 2)
+            return launch_pair<128, 4, 2, LAYOUT, 2>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
         if (c.bn == 192 && c.stages == 3 && c.ks == 2 && c.wg == 3)
             return launch_pair<192, 3, 2, LAYOUT, 3>(A, a_rows, B, b_rows, p, 2 * grid_pairs, stream);
         return DG_ERR_UNSUPPORTED;
@@ -702,7 +716,7 @@ dg_status_t dense_gemm(const void *A, const float *sA, const void *B, const floa
     p.num_kb = K / 128;
     p.nbn = (N + 127) / 128;
     p.num_mb = (M + 127) / 128;
-    p.raster = choose_raster(p.num_mb);
+    p.raster = choose_raster(p.num_mb, dg::kBM, K);
     p.timeout_ns = g_timeout_ns.load();
     p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
@@ -839,7 +853,10 @@ dg_status_t launch_bs(const void *A, uint64_t a_rows, const void *B, uint64_t b_
         attr_set[dev].store(true);
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    // the K split runs a 3-D grid (split, column tile, 128-row block)
+    cfg.gridDim = SPLIT ? dim3(static_cast<unsigned>(p.ksplit), static_cast<unsigned>(p.num_nb),
+                               static_cast<unsigned>(p.num_mb))
+                        : dim3(static_cast<unsigned>(grid), 1, 1);
     cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cfg.stream = stream;
@@ -923,7 +940,7 @@ dg_status_t dispatch_bs(const BsChoice &c, const void *A, uint64_t a_rows, const
         // the pair scheduler counts 256-row pair rows
         p.num_mb = (p.num_mb + 1) / 2;
         if (LAYOUT != dg::kMasked)
-            p.raster = choose_raster(p.num_mb);
+            p.raster = choose_raster(p.num_mb, 2 * dg::kBM, p.K);
         const int pairs = sms / 2;
         const int64_t ptiles = static_cast<int64_t>(p.num_mb) * p.num_nb;
         int grid_pairs = pairs;
@@ -988,7 +1005,7 @@ GemmParams bs_params(const int32_t *sfa, const int32_t *sfb, void *D, int M, int
     p.num_kg = (p.num_kb + 3) / 4;
     p.nbn = (N + 127) / 128;
     p.num_mb = (M + 127) / 128;
-    p.raster = choose_raster(p.num_mb);
+    p.raster = choose_raster(p.num_mb, dg::kBM, K);
     p.timeout_ns = g_timeout_ns.load();
     p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
@@ -1119,7 +1136,7 @@ dg_status_t dg_fp8_gemm_nt_acc(const void *A, const float *sA, const void *B, co
     p.num_kb = K / 128;
     p.nbn = (N + 127) / 128;
     p.num_mb = (M + 127) / 128;
-    p.raster = choose_raster(p.num_mb);
+    p.raster = choose_raster(p.num_mb, dg::kBM, K);
     p.timeout_ns = g_timeout_ns.load();
     p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
@@ -1166,7 +1183,7 @@ dg_status_t dg_fp8_grouped_gemm_contiguous(const void *A, const float *sA, const
     p.num_kb = K / 128;
     p.nbn = (N + 127) / 128;
     p.num_mb = M_total / 128;
-    p.raster = choose_raster(p.num_mb);
+    p.raster = choose_raster(p.num_mb, dg::kBM, K);
     p.timeout_ns = g_timeout_ns.load();
     p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
@@ -1218,9 +1235,15 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const voi
     p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();
     const int em = (expected_m > 0 && expected_m < max_m) ? expected_m : max_m;
-    const Plan plan = choose_plan(static_cast<int64_t>(num_groups) * ((em + 127) / 128),
-                                  static_cast<int64_t>(num_groups) * ((em + 255) / 256), N,
-                                  p.num_kb, sms, false);
+    Plan plan = choose_plan(static_cast<int64_t>(num_groups) * ((em + 127) / 128),
+                            static_cast<int64_t>(num_groups) * ((em + 255) / 256), N, p.num_kb, sms, false);
+    // Decode-sized groups (at most two 128-row blocks each) make the problem
+    // HBM-bound on the weights: the 128-column one-CTA tile with its five
+    // one-K-block stages keeps the most weight bytes in flight per SM and
+    // measured best (16 x 256 x 4096 x 7168: 165 us against 171-176 us for
+    // 112, 224 and 256 columns), unless a tile width or family is pinned.
+    if (em <= 2 * dg::kBM && forced_block_n() <= 0 && forced_pair() < 0)
+        plan = Plan{kTileChoices[1], 1};
     if (print_configs())
         std::fprintf(stderr,
                      "[dg] masked G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d sms=%d\n",
@@ -1468,7 +1491,9 @@ int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, i
         m_blocks *= groups;
         pair_rows *= groups;
     }
-    const Plan plan = choose_plan(m_blocks, pair_rows, N, K / 128 > 0 ? K / 128 : 1, sms, layout == 0);
+    Plan plan = choose_plan(m_blocks, pair_rows, N, K / 128 > 0 ? K / 128 : 1, sms, layout == 0);
+    if (layout == 2 && M <= 2 * dg::kBM && forced_block_n() <= 0 && forced_pair() < 0)
+        plan = Plan{kTileChoices[1], 1};  // as dg_fp8_grouped_gemm_masked: decode-sized groups
     const TileChoice &c = plan.c;
     return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
                          "layout=%d BM=%d BN=%d BK=128 stages=%d ks=%d ksplit=%d pair=%d wg=%d sms=%d m_blocks=%lld n_blocks=%d",
@@ -1599,7 +1624,7 @@ extern "C" dg_status_t dg_fp8_gemm_nt_noalloc(const void *A, const float *sA, co
     p.nbn = (N + 127) / 128;
     p.num_mb = (M + 127) / 128;
     p.num_nb = (N + kBN - 1) / kBN;
-    p.raster = choose_raster(p.num_mb);
+    p.raster = choose_raster(p.num_mb, dg::kBM, K);
     p.timeout_ns = g_timeout_ns.load();
     p.stamps = g_stamps.load();
     p.stall_injection = g_stall_injection.load();

@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
                        const __grid_constant__ CUtensorMap tmap_drem, const GemmParams p)
 {
     using Cfg = BsConfig<BN, STAGES, KS, PAIR, SPLIT>;
-    using Sched = std::conditional_t<PAIR, PairScheduler<LAYOUT>, TileScheduler<LAYOUT>>;
+    using Sched = std::conditional_t<PAIR, PairScheduler<LAYOUT>, TileScheduler<LAYOUT, SPLIT>>;
     static_assert(LAYOUT == kDense || LAYOUT == kContiguous || LAYOUT == kMasked,
                   "block-scaled mode: dense, contiguous and masked layouts");
     static_assert(!SPLIT || LAYOUT == kDense, "the K split is implemented for the dense layout");
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
         Sched sched(p);
         TileCoord tc;
         uint32_t stage = 0, phase = 0, issued = 0;
-        bool ok = !(p.stall_injection && blockIdx.x < CTAS);
+        bool ok = !(p.stall_injection && blockIdx.x < CTAS && blockIdx.y == 0 && blockIdx.z == 0);
         while (ok && sched.next(tc, is_a && leader && lane == 0)) {
             const int row = is_a ? (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * TILE_ROWS +
                                        static_cast<int>(rank) * kBM
@@ -656,13 +656,22 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
                 const int lr = it % rows_per;  // rows fastest: contiguous reads
                 const int c4 = it / rows_per;
                 const int r = static_cast<int>(rank_s) * rows_per + lr;
+                // all S loads in flight at once (S <= 16), then the sum in
+                // split order
+                float4 w[16];
+#pragma unroll
+                for (int src = 0; src < 16; ++src)
+                    if (src < S)
+                        w[src] = __ldcg(src0 + (static_cast<size_t>(src) * C4 + c4) * kBM + r);
                 float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int src = 0; src < S; ++src) {
-                    const float4 w = __ldcg(src0 + (static_cast<size_t>(src) * C4 + c4) * kBM + r);
-                    sum.x += w.x;
-                    sum.y += w.y;
-                    sum.z += w.z;
-                    sum.w += w.w;
+#pragma unroll
+                for (int src = 0; src < 16; ++src) {
+                    if (src < S) {
+                        sum.x += w[src].x;
+                        sum.y += w[src].y;
+                        sum.z += w[src].z;
+                        sum.w += w[src].w;
+                    }
                 }
                 const int grow = tc.mb * kBM + r;
                 const int gcol = tc.nb * BN + c4 * 4;

@@ -72,8 +72,9 @@ static __device__ unsigned int g_status_word = 0;
 
 __device__ __forceinline__ void record_status(uint32_t code, uint32_t role, uint32_t stage)
 {
-    const uint32_t w = (code & 0xFF) | ((role & 0xF) << 8) | ((stage & 0xFF) << 12) |
-                       ((blockIdx.x & 0xFFF) << 20);
+    // the CTA's linear index (the K-split kernels run a 3-D grid)
+    const uint32_t cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    const uint32_t w = (code & 0xFF) | ((role & 0xF) << 8) | ((stage & 0xFF) << 12) | ((cta & 0xFFF) << 20);
     atomicCAS(&g_status_word, 0u, w);
 }
 
@@ -179,8 +180,11 @@ __device__ __forceinline__ bool padding_block_has_rows(const int32_t *m_indices,
 }
 
 // Enumerates this CTA's tiles: t = blockIdx.x, blockIdx.x + gridDim.x, ...
-// Every role runs its own copy and sees the same sequence.
-template <int LAYOUT>
+// Every role runs its own copy and sees the same sequence.  With SPLIT (the
+// K-split kernels) the grid is 3-D -- x the split (a cluster of ksplit CTAs
+// along x), y the column tile, z the 128-row block -- and each CTA has
+// exactly one tile, so no index needs a division.
+template <int LAYOUT, bool SPLIT = false>
 struct TileScheduler {
     const GemmParams &p;
     int next_t;
@@ -188,29 +192,35 @@ struct TileScheduler {
 
     int stride;
 
-    // With a K split, the ksplit CTAs of a cluster share one tile (and the
-    // grid holds exactly one tile per cluster).
     __device__ explicit TileScheduler(const GemmParams &params)
-        : p(params), next_t(blockIdx.x / params.ksplit), stride(gridDim.x / params.ksplit) {}
+        : p(params), next_t(SPLIT ? 0 : static_cast<int>(blockIdx.x)), stride(SPLIT ? 1 : static_cast<int>(gridDim.x)) {}
 
     // This CTA's K blocks: [begin, end).
     __device__ int kb_begin() const
     {
         if constexpr (LAYOUT == kKGrouped)
             return cur_kb0;
-        return p.ksplit > 1 ? static_cast<int>(blockIdx.x % p.ksplit) * p.kb_per_split : 0;
+        return SPLIT ? static_cast<int>(blockIdx.x) * p.kb_per_split : 0;
     }
     __device__ int kb_end() const
     {
         if constexpr (LAYOUT == kKGrouped)
             return cur_kb1;
-        return p.ksplit > 1 ? min(p.num_kb, kb_begin() + p.kb_per_split) : p.num_kb;
+        return SPLIT ? min(p.num_kb, kb_begin() + p.kb_per_split) : p.num_kb;
     }
     int cur_kb0 = 0, cur_kb1 = 0;  // K-grouped: the current tile's K blocks
 
     __device__ bool next(TileCoord &tc, bool report)
     {
-        if constexpr (LAYOUT == kKGrouped) {
+        if constexpr (SPLIT) {
+            static_assert(LAYOUT == kDense, "the K split is implemented for the dense layout");
+            if (next_t++ > 0)
+                return false;
+            tc.g = 0;
+            tc.nb = static_cast<int>(blockIdx.y);
+            tc.mb = static_cast<int>(blockIdx.z);
+            return true;
+        } else if constexpr (LAYOUT == kKGrouped) {
             // tiles group by group, each group's m-blocks fastest
             const int per_group = p.num_mb * p.num_nb;
             const int t = next_t;
@@ -294,12 +304,11 @@ struct TileScheduler {
 
 // ----------------------------------------------------------- bounded waits
 
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
-                                             volatile int *abort_flag, uint32_t role,
-                                             uint32_t stage, bool honour_abort)
+// The spin loop of a wait that did not complete at once.
+__device__ __forceinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                               volatile int *abort_flag, uint32_t role, uint32_t stage,
+                                               bool honour_abort)
 {
-    if (mbar_try_wait(bar, parity))
-        return true;
     const uint64_t t0 = global_timer_ns();
     uint32_t spins = 0;
     while (true) {
@@ -315,6 +324,15 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint
             }
         }
     }
+}
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                             volatile int *abort_flag, uint32_t role,
+                                             uint32_t stage, bool honour_abort)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    return wait_bounded_slow(bar, parity, timeout_ns, abort_flag, role, stage, honour_abort);
 }
 
 // Lane 0 waits, the whole warp gets the outcome.
@@ -392,7 +410,7 @@ struct KernelConfig {
     static_assert(BN % NUM_WG == 0 && BN_WG % 4 == 0, "promotion columns per warpgroup: a multiple of 4");
     static_assert(BN_WG % 8 == 0 || (SPLIT && !COLSCALE && BN_WG == RMAX),
                   "a column count that is not a multiple of 8 is read in one round and split-reduced");
-    static_assert(NUM_WG * 4 + 2 <= 32 && NUM_WG <= 14, "warps per CTA; named barriers 1..NUM_WG");
+    static_assert(NUM_WG * 4 + 2 <= 32 && NUM_WG <= 14, "warps per CTA; named barriers 1..NUM_WG, 15 at start-up");
     static_assert(BN_WG <= 128, "a warpgroup's columns must span at most two 128-wide sB blocks");
     static_assert(NBUF >= 2, "double-buffered TMEM at least");
     static_assert(B_BYTES % 1024 == 0, "B tiles must keep 1024-byte swizzle atoms aligned");
@@ -404,22 +422,21 @@ struct KernelConfig {
 
 // Loads COLS (multiple of 8, may be 0) consecutive TMEM columns of this
 // warp's 32 lanes into r[0..COLS).
-template <int COLS>
+// The column offsets are compile-time constants (recursion on Q), so r stays
+// in registers.
+template <int COLS, int Q = 0>
 __device__ __forceinline__ void tmem_load_cols(uint32_t taddr, uint32_t *r)
 {
     static_assert(COLS % 4 == 0, "TMEM loads of whole 4-column groups");
-#pragma unroll
-    for (int q = 0; q < COLS;) {
-        if (q + 16 <= COLS) {
-            tmem_ld_32x32b_x16(taddr + q, *reinterpret_cast<uint32_t(*)[16]>(r + q));
-            q += 16;
-        } else if (q + 8 <= COLS) {
-            tmem_ld_32x32b_x8(taddr + q, *reinterpret_cast<uint32_t(*)[8]>(r + q));
-            q += 8;
-        } else {
-            tmem_ld_32x32b_x4(taddr + q, *reinterpret_cast<uint32_t(*)[4]>(r + q));
-            q += 4;
-        }
+    if constexpr (Q + 16 <= COLS) {
+        tmem_ld_32x32b_x16(taddr + Q, *reinterpret_cast<uint32_t(*)[16]>(r + Q));
+        tmem_load_cols<COLS, Q + 16>(taddr, r);
+    } else if constexpr (Q + 8 <= COLS) {
+        tmem_ld_32x32b_x8(taddr + Q, *reinterpret_cast<uint32_t(*)[8]>(r + Q));
+        tmem_load_cols<COLS, Q + 8>(taddr, r);
+    } else if constexpr (Q + 4 <= COLS) {
+        tmem_ld_32x32b_x4(taddr + Q, *reinterpret_cast<uint32_t(*)[4]>(r + Q));
+        tmem_load_cols<COLS, Q + 4>(taddr, r);
     }
 }
 
@@ -482,35 +499,45 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
     const int lane = threadIdx.x % 32;
     stamp_start(p);
 
-    if (warp == Cfg::PRODUCER_WARP && lane == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            // full: the elected producer lane's expect-tx arrival plus one
-            // cp.async arrival from each of the 32 producer lanes
-            mbar_init(smem_addr(full_bar + s), 1 + 32);
-            mbar_init(smem_addr(empty_bar + s), 1);
-            mbar_init(smem_addr(sread_bar + s), Cfg::NUM_PROMO_WARPS);
+    // Start-up.  The producer warp does not wait for the TMEM allocation:
+    // once its lane 0 has initialised the barriers, the warp arrives on the
+    // start barrier and begins issuing loads; every other warp waits there
+    // until the barriers exist and TMEM is allocated.
+    constexpr uint32_t kStartBarrier = 15;
+    if (warp == Cfg::PRODUCER_WARP) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmap_a);
+            tma_prefetch_desc(&tmap_b);
+            for (int s = 0; s < STAGES; ++s) {
+                // full: the elected producer lane's expect-tx arrival plus one
+                // cp.async arrival from each of the 32 producer lanes
+                mbar_init(smem_addr(full_bar + s), 1 + 32);
+                mbar_init(smem_addr(empty_bar + s), 1);
+                mbar_init(smem_addr(sread_bar + s), Cfg::NUM_PROMO_WARPS);
+            }
+            for (int b = 0; b < NBUF; ++b) {
+                mbar_init(smem_addr(tfull_bar + b), 1);
+                mbar_init(smem_addr(tempty_bar + b), Cfg::NUM_PROMO_WARPS);
+            }
+            *abort_flag = 0;
+            fence_barrier_init();
+            if (Cfg::EPI_FULL_BOXES > 0)
+                tma_prefetch_desc(&tmap_d64);
+            if (Cfg::EPI_REM > 0)
+                tma_prefetch_desc(&tmap_drem);
         }
-        for (int b = 0; b < NBUF; ++b) {
-            mbar_init(smem_addr(tfull_bar + b), 1);
-            mbar_init(smem_addr(tempty_bar + b), Cfg::NUM_PROMO_WARPS);
+        __syncwarp();
+        named_barrier_arrive(kStartBarrier, Cfg::THREADS);
+    } else {
+        if (warp == Cfg::MMA_WARP) {
+            tmem_alloc(smem_addr(tmem_slot), Cfg::TMEM_COLS);
+            tmem_relinquish_alloc_permit();
         }
-        *abort_flag = 0;
-        fence_barrier_init();
-        tma_prefetch_desc(&tmap_a);
-        tma_prefetch_desc(&tmap_b);
-        if (Cfg::EPI_FULL_BOXES > 0)
-            tma_prefetch_desc(&tmap_d64);
-        if (Cfg::EPI_REM > 0)
-            tma_prefetch_desc(&tmap_drem);
+        tc_fence_before_sync();
+        named_barrier_sync(kStartBarrier, Cfg::THREADS);
+        tc_fence_after_sync();
     }
-    if (warp == Cfg::MMA_WARP) {
-        tmem_alloc(smem_addr(tmem_slot), Cfg::TMEM_COLS);
-        tmem_relinquish_alloc_permit();
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_base = warp == Cfg::PRODUCER_WARP ? 0u : *tmem_slot;
     const uint64_t tmo = p.timeout_ns;
     // Waits for this CTA's own copies and MMAs in flight before it exits use
     // at least a second, however short the pipeline limit is set.
@@ -522,13 +549,13 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
         // lane issues the two operand boxes of a stage; every lane copies a
         // 16-byte piece of each K block's LHS scales, and lanes 0-2 copy the
         // weight-block scales, all landing on the stage's full barrier.
-        TileScheduler<LAYOUT> sched(p);
+        TileScheduler<LAYOUT, SPLIT> sched(p);
         TileCoord tc;
         uint32_t stage = 0, phase = 0;
         uint32_t issued = 0;
         // Test hook (dg_set_stall_injection): CTA 0 never fills a stage, so
         // its consumers' waits run out and report DG_ERR_TIMEOUT.
-        bool ok = !(p.stall_injection && blockIdx.x == 0);
+        bool ok = !(p.stall_injection && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0);
         while (ok && sched.next(tc, lane == 0)) {
             const int a_row = (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * kBM;
             // (the K-grouped layout shares one B across its groups)
@@ -623,7 +650,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
         // ------------------------------------------------------- MMA issuer
         // Uniform loop; the descriptors stay warp-uniform and one elected
         // lane issues the MMAs and the commits.
-        TileScheduler<LAYOUT> sched(p);
+        TileScheduler<LAYOUT, SPLIT> sched(p);
         TileCoord tc;
         uint32_t stage = 0, phase = 0, acc_i = 0;
         // the most recent commit (barrier, phase parity): it fires once
@@ -703,7 +730,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
         const int row = quad * 32 + lane;  // tile row == TMEM lane
         const int wg_tid = threadIdx.x % 128;
         const uint32_t lane_bits = static_cast<uint32_t>(quad * 32) << 16;
-        TileScheduler<LAYOUT> sched(p);
+        TileScheduler<LAYOUT, SPLIT> sched(p);
         TileCoord tc;
         uint32_t acc_i = 0, stage = 0, phase = 0;
         bool ok = true;
@@ -959,7 +986,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
         // on timing), then rounds to bf16.
         const int S = p.ksplit;
         const uint32_t rank = cluster_ctarank();
-        TileScheduler<LAYOUT> sched(p);
+        TileScheduler<LAYOUT, SPLIT> sched(p);
         TileCoord tc;
         if (sched.next(tc, false)) {
             // rows [r0, r1) of the tile: S need not divide 128
@@ -972,13 +999,22 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
                 const int lr = it % rows_per;  // rows fastest: contiguous reads
                 const int c4 = it / rows_per;
                 const int r = r0 + lr;
+                // all S loads in flight at once (S <= 16), then the sum in
+                // split order
+                float4 v[16];
+#pragma unroll
+                for (int src = 0; src < 16; ++src)
+                    if (src < S)
+                        v[src] = __ldcg(src0 + (static_cast<size_t>(src) * C4 + c4) * kBM + r);
                 float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int src = 0; src < S; ++src) {
-                    const float4 v = __ldcg(src0 + (static_cast<size_t>(src) * C4 + c4) * kBM + r);
-                    sum.x += v.x;
-                    sum.y += v.y;
-                    sum.z += v.z;
-                    sum.w += v.w;
+#pragma unroll
+                for (int src = 0; src < 16; ++src) {
+                    if (src < S) {
+                        sum.x += v[src].x;
+                        sum.y += v[src].y;
+                        sum.z += v[src].z;
+                        sum.w += v[src].w;
+                    }
                 }
                 const int grow = tc.mb * kBM + r;
                 const int gcol = tc.nb * BN + c4 * 4;

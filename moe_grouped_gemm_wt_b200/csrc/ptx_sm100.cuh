@@ -273,6 +273,14 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Arrives on named barrier `id` (expecting `count` threads) without waiting:
+// the memory operations of this thread before it are visible to the threads
+// that wait on the barrier (bar.sync) once it completes.
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // AND of `pred` over the `count` threads (multiple of 32) that reach named
 // barrier `id`; also a barrier among them.
 __device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t count, bool pred)
