@@ -63,9 +63,9 @@ EncodeTiledFn encode_fn()
 // enter the key: the encoded map holds only the address and the layout.
 struct TmapKey {
     const void *base;
-    uint64_t dims[3];
-    uint64_t strides[2];
-    uint32_t box[3];
+    uint64_t dims[4];
+    uint64_t strides[3];
+    uint32_t box[4];
     uint32_t rank, dtype, swizzle, promo;
     bool operator==(const TmapKey &o) const { return std::memcmp(this, &o, sizeof(*this)) == 0; }
 };
@@ -114,7 +114,7 @@ bool encode_cached(CUtensorMap *map, CUtensorMapDataType dtype, uint32_t rank, c
     EncodeTiledFn enc = encode_fn();
     if (!enc)
         return false;
-    cuuint32_t estr[3] = {1, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
     if (enc(map, dtype, rank, const_cast<void *>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
@@ -161,6 +161,21 @@ bool make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t
     cuuint32_t box[2] = {box_inner, box_rows};
     return encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, swizzle,
                          CU_TENSOR_MAP_L2_PROMOTION_NONE);
+}
+
+// The K-split workspace [tiles][S][BN/4][128] float4s viewed in 4-D as
+// (float within a column quad's 128 rows, column quad, split, tile), with a
+// box of one CTA's rows_per rows of every column quad and split of one tile.
+bool make_tmap_split_ws(CUtensorMap *map, const float *ws, int bn, int S, uint64_t tiles, int rows_per)
+{
+    const uint64_t c4 = static_cast<uint64_t>(bn / 4);
+    cuuint64_t dims[4] = {4ull * 128ull, c4, static_cast<uint64_t>(S), tiles};
+    cuuint64_t strides[3] = {4ull * 128ull * 4ull, 4ull * 128ull * 4ull * c4,
+                             4ull * 128ull * 4ull * c4 * static_cast<uint64_t>(S)};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(4 * rows_per), static_cast<cuuint32_t>(c4),
+                         static_cast<cuuint32_t>(S), 1};
+    return encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ws, dims, strides, box,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 // ------------------------------------------------------------------- device
@@ -239,12 +254,18 @@ struct TileChoice {
     double tile_us;  // per-tile fill, drain and epilogue (cost model, us)
     int wg = 2;      // promotion warpgroups
     int rebal = 0;   // pair tiles: registers rebalanced with setmaxnreg (always for wg >= 3)
+    int masked_only = 0;  // taken only by the masked layout's decode-sized groups
 };
 constexpr TileChoice kTileChoices[] = {
     {112, 3, 2, 0, 0.41, 0, 1.9}, {128, 5, 1, 0, 0.53, 0, 1.9}, {224, 2, 2, 0, 0.78, 0, 1.9},
     {256, 3, 1, 0, 0.68, 0, 1.9}, {144, 3, 2, 1, 0.40, 0, 1.9, 3}, {160, 3, 2, 0, 0.441, 1, 2.2},
-    {192, 3, 2, 0, 0.50, 1, 2.2, 3},
+    {192, 3, 2, 0, 0.50, 1, 2.2, 3}, {128, 3, 2, 0, 0.50, 0, 1.9, 2, 0, 1},
 };
+// The masked layout's tile for decode-sized groups (at most two 128-row
+// blocks per group): HBM-bound on the weights, it keeps six K blocks in
+// flight per SM in three stages of two-K-block boxes (half the TMA
+// instructions of one-K-block stages) and stores rows directly.
+constexpr int kMaskedDecodeTile = 7;
 constexpr int kSplitFixedNs = 1500;  // cluster reduction + pipeline fill of a split CTA
 
 // Tile width pinned by dg_set_block_n (0 = the cost model decides); its
@@ -331,6 +352,8 @@ Plan choose_plan(int64_t m_blocks, int64_t pair_rows, int N, int num_kb, int sms
         if ((limits & kWholeBoxes) && c.bn % 128 != 0)
             continue;
         if (forced_pair() >= 0 && c.pair != forced_pair())
+            continue;
+        if (c.masked_only)
             continue;
         if (c.pair) {
             const int pairs = sms / 2;
@@ -423,6 +446,16 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
             return DG_ERR_CUDA;
     } else {
         tdrem = td64;
+    }
+    if (SPLIT && p.D != nullptr && p.ksplit >= 2 && dg::kBM % p.ksplit == 0) {
+        // the K-split reduction's maps: the partials (in place of the
+        // epilogue's 64-column boxes) and one CTA's output rows
+        const int rows_per = dg::kBM / p.ksplit;
+        const uint64_t tiles = static_cast<uint64_t>(p.num_mb) * static_cast<uint64_t>(p.num_nb);
+        if (!make_tmap_split_ws(&td64, p.ws, BN, p.ksplit, tiles, rows_per) ||
+            !make_tmap_bf16(&tdrem, p.D, static_cast<uint64_t>(p.N), d_rows, BN, rows_per,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+            return DG_ERR_CUDA;
     }
     auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT, SPLIT, A_MN, B_MN, NWG>;
     static std::atomic<bool> attr_set[kMaxDevices];
@@ -662,6 +695,9 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
     DG_TILE_CASE(128, 5, 1)
     DG_TILE_CASE(224, 2, 2)
     DG_TILE_CASE(256, 3, 1)
+    if constexpr (LAYOUT == dg::kMasked) {
+        DG_TILE_CASE(128, 3, 2)
+    }
 #undef DG_TILE_CASE
     if constexpr (LAYOUT == dg::kDense && !B_MN) {
         if (c.bn == 144 && c.stages == 3 && c.ks == 2 && c.split && c.wg == 3)
@@ -1238,12 +1274,14 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const voi
     Plan plan = choose_plan(static_cast<int64_t>(num_groups) * ((em + 127) / 128),
                             static_cast<int64_t>(num_groups) * ((em + 255) / 256), N, p.num_kb, sms, false);
     // Decode-sized groups (at most two 128-row blocks each) make the problem
-    // HBM-bound on the weights: the 128-column one-CTA tile with its five
-    // one-K-block stages keeps the most weight bytes in flight per SM and
-    // measured best (16 x 256 x 4096 x 7168: 165 us against 171-176 us for
-    // 112, 224 and 256 columns), unless a tile width or family is pinned.
+    // HBM-bound on the weights: the 128-column one-CTA tile with three
+    // stages of two K blocks keeps six K blocks in flight per SM with half
+    // the TMA instructions of one-K-block stages, and measured best
+    // (16 x 256 x 4096 x 7168: 156 us, against 172 us for five one-K-block
+    // stages and 171-176 us for 112, 224 and 256 columns), unless a tile
+    // width or family is pinned.
     if (em <= 2 * dg::kBM && forced_block_n() <= 0 && forced_pair() < 0)
-        plan = Plan{kTileChoices[1], 1};
+        plan = Plan{kTileChoices[kMaskedDecodeTile], 1};
     if (print_configs())
         std::fprintf(stderr,
                      "[dg] masked G=%d max_m=%d expected_m=%d N=%d K=%d -> BM=%d BN=%d stages=%d ks=%d sms=%d\n",
@@ -1493,7 +1531,7 @@ int dg_describe_config(int layout, int M, int N, int K, int groups, char *buf, i
     }
     Plan plan = choose_plan(m_blocks, pair_rows, N, K / 128 > 0 ? K / 128 : 1, sms, layout == 0);
     if (layout == 2 && M <= 2 * dg::kBM && forced_block_n() <= 0 && forced_pair() < 0)
-        plan = Plan{kTileChoices[1], 1};  // as dg_fp8_grouped_gemm_masked: decode-sized groups
+        plan = Plan{kTileChoices[kMaskedDecodeTile], 1};  // as dg_fp8_grouped_gemm_masked: decode-sized groups
     const TileChoice &c = plan.c;
     return std::snprintf(buf, len > 0 ? static_cast<size_t>(len) : 0,
                          "layout=%d BM=%d BN=%d BK=128 stages=%d ks=%d ksplit=%d pair=%d wg=%d sms=%d m_blocks=%lld n_blocks=%d",

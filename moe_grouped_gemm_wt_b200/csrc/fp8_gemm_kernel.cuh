@@ -388,7 +388,13 @@ struct KernelConfig {
     static constexpr int ACC_STRIDE = (BN + 31) / 32 * 32;
     static constexpr int NBUF = (512 / ACC_STRIDE) < 4 ? (512 / ACC_STRIDE) : 4;
     static constexpr int TMEM_COLS = NBUF * ACC_STRIDE <= 256 ? 256 : 512;
-    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 2 * NBUF) + 16;
+    // + one barrier for the K-split reduction's TMA load
+    static constexpr int BAR_BYTES = 8 * (3 * STAGES + 2 * NBUF + 1) + 16;
+    // K split: the reduction reads this CTA's rows of all S partials
+    // (BN/4 x 128 float4s whatever S is) into the idle operand ring at
+    // offset 0, and stages its bf16 rows (at most 64 x BN) after them.
+    static constexpr int RED_IN_BYTES = (BN / 4) * kBM * 16;
+    static constexpr int RED_OUT_OFFSET = (RED_IN_BYTES + 1023) / 1024 * 1024;
     // Epilogue: each promotion warpgroup stages its 128 rows of the output in
     // shared memory one box at a time and TMA-stores it: boxes of 64 columns
     // (128-byte rows, 128-byte swizzle) and one remainder box.
@@ -399,12 +405,15 @@ struct KernelConfig {
     static constexpr int EPI_OFFSET = (PIPE_BYTES + BAR_BYTES + 1023) / 1024 * 1024;
     // One staging buffer per output box when shared memory allows, so a
     // warpgroup stores all its boxes without waiting for an earlier store to
-    // finish reading its buffer; else one buffer reused box after box.
+    // finish reading its buffer; else one buffer reused box after box.  A
+    // ring too deep for even one buffer per warpgroup (the masked decode
+    // tile) stores every row segment directly (EPI_STAGED false).
     static constexpr int EPI_BOXES = EPI_FULL_BOXES + (EPI_REM > 0 ? 1 : 0);
+    static constexpr bool EPI_STAGED = 1024 + EPI_OFFSET + NUM_WG * EPI_WG_BYTES <= 232448;
     static constexpr int EPI_BUFS =
         1024 + EPI_OFFSET + NUM_WG * EPI_BOXES * EPI_WG_BYTES <= 232448 ? EPI_BOXES : 1;
     static constexpr int SMEM_BYTES =
-        1024 /*align slack*/ + EPI_OFFSET + (SPLIT ? 0 : NUM_WG * EPI_BUFS * EPI_WG_BYTES);
+        1024 /*align slack*/ + EPI_OFFSET + ((SPLIT || !EPI_STAGED) ? 0 : NUM_WG * EPI_BUFS * EPI_WG_BYTES);
 
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128: multiple of 16, <= 256");
     static_assert(BN % NUM_WG == 0 && BN_WG % 4 == 0, "promotion columns per warpgroup: a multiple of 4");
@@ -418,6 +427,8 @@ struct KernelConfig {
     static_assert(EPI_REM % 8 == 0, "remainder box must be whole 16-byte chunks");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
     static_assert(!SPLIT || BN_WG % 4 == 0, "split reduction works on float4 columns");
+    static_assert(!SPLIT || RED_OUT_OFFSET + 64 * BN * 2 <= STAGES * STAGE_BYTES,
+                  "the split reduction's buffers fit in the operand ring");
 };
 
 // Loads COLS (multiple of 8, may be 0) consecutive TMEM columns of this
@@ -491,7 +502,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
     uint64_t *sread_bar = bars + 2 * STAGES;   // promotion warps have read the stage's scales
     uint64_t *tfull_bar = bars + 3 * STAGES;   // TMEM partial buffer written
     uint64_t *tempty_bar = bars + 3 * STAGES + NBUF;  // TMEM partial buffer read out
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 2 * NBUF);
+    uint64_t *red_bar = bars + 3 * STAGES + 2 * NBUF;  // K split: the reduction's partials landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(red_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     uint8_t *epi_stage = smem + Cfg::EPI_OFFSET;  // 1024-byte aligned, EPI_BUFS buffers per warpgroup
 
@@ -519,11 +531,14 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
                 mbar_init(smem_addr(tfull_bar + b), 1);
                 mbar_init(smem_addr(tempty_bar + b), Cfg::NUM_PROMO_WARPS);
             }
+            mbar_init(smem_addr(red_bar), 1);
             *abort_flag = 0;
             fence_barrier_init();
-            if (Cfg::EPI_FULL_BOXES > 0)
+            // (K split: tmap_d64 describes the partials, tmap_drem the
+            // reduction's output rows)
+            if (SPLIT || Cfg::EPI_FULL_BOXES > 0)
                 tma_prefetch_desc(&tmap_d64);
-            if (Cfg::EPI_REM > 0)
+            if (SPLIT || Cfg::EPI_REM > 0)
                 tma_prefetch_desc(&tmap_drem);
         }
         __syncwarp();
@@ -919,7 +934,7 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
                                          col0, p.N);
                 continue;
             }
-            const bool tile_rows_ok = named_barrier_and(
+            const bool tile_rows_ok = Cfg::EPI_STAGED && named_barrier_and(
                 1 + wg, 128, LAYOUT == kDense ? (tc.mb * kBM < p.M) : row_ok);
             if (tile_rows_ok) {
                 const int grow0 = (LAYOUT == kMasked ? tc.g * p.M : 0) + tc.mb * kBM;
@@ -995,6 +1010,55 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
             constexpr int C4 = BN / 4;
             const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
             const float4 *src0 = reinterpret_cast<const float4 *>(p.ws) + tile * S * C4 * kBM;
+            if (p.D32 == nullptr && kBM % S == 0) {
+                // bf16 output.  One TMA box brings this CTA's rows of all S
+                // partials, [S][C4][rows_per] float4s, into the idle operand
+                // ring; the sums (in split order, as below) are rounded,
+                // staged as [rows_per][BN] bf16 and stored with one TMA box
+                // (rows past M and columns past N are clipped).
+                const float4 *red_in = reinterpret_cast<const float4 *>(smem);
+                uint8_t *red_out = smem + Cfg::RED_OUT_OFFSET;
+                if (threadIdx.x == 0) {
+                    // the partials were written by generic-proxy stores
+                    fence_proxy_async_global();
+                    mbar_arrive_expect_tx(smem_addr(red_bar), Cfg::RED_IN_BYTES);
+                    tma_load_4d(smem_addr(smem), &tmap_d64, smem_addr(red_bar), 4 * r0, 0, 0,
+                                static_cast<int>(tile));
+                }
+                // the box must land whatever the abort flag says: this CTA's
+                // shared memory may not be left while the copy is in flight
+                int got_lane = 0;
+                if (lane == 0)
+                    got_lane = wait_bounded(smem_addr(red_bar), 0, drain_tmo, abort_flag, kRoleDrain, 40, false)
+                                   ? 1 : 0;
+                const bool got = __shfl_sync(0xFFFFFFFFu, got_lane, 0) != 0;
+                if (got) {
+                    for (int it = threadIdx.x; it < rows_per * C4; it += Cfg::THREADS) {
+                        const int lr = it % rows_per;  // rows fastest: conflict-free reads
+                        const int c4 = it / rows_per;
+                        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int src = 0; src < S; ++src) {
+                            const float4 v = red_in[(src * C4 + c4) * rows_per + lr];
+                            sum.x += v.x;
+                            sum.y += v.y;
+                            sum.z += v.z;
+                            sum.w += v.w;
+                        }
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
+                        uint2 u;
+                        u.x = *reinterpret_cast<uint32_t *>(&h0);
+                        u.y = *reinterpret_cast<uint32_t *>(&h1);
+                        *reinterpret_cast<uint2 *>(red_out + (lr * BN + 4 * c4) * 2) = u;
+                    }
+                }
+                fence_proxy_async_smem();
+                if (__syncthreads_and(got ? 1 : 0) && threadIdx.x == 0) {
+                    tma_store_2d(&tmap_drem, smem_addr(red_out), tc.nb * BN, tc.mb * kBM + r0);
+                    bulk_commit_group();
+                    bulk_wait_group<0>();
+                }
+            } else
             for (int it = threadIdx.x; it < rows_per * C4; it += Cfg::THREADS) {
                 const int lr = it % rows_per;  // rows fastest: contiguous reads
                 const int c4 = it / rows_per;

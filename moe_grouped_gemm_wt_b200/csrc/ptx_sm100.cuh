@@ -176,6 +176,24 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
+// 4-D tiled load (x innermost).
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *tmap, uint32_t bar, int x,
+                                            int y, int z, int w)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
+
+// Orders this thread's generic-proxy accesses to global memory before its
+// later async-proxy (TMA) accesses, and the reverse.
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // 3-D tiled load for a CTA pair (cta_group::2): the box lands in this CTA's
 // shared memory at `dst`, and its transaction bytes are signalled on
 // `bar_cluster`, a barrier of either CTA of the pair given by its
