@@ -264,7 +264,8 @@ constexpr TileChoice kTileChoices[] = {
 // The masked layout's tile for decode-sized groups (at most two 128-row
 // blocks per group): HBM-bound on the weights, it keeps six K blocks in
 // flight per SM in three stages of two-K-block boxes (half the TMA
-// instructions of one-K-block stages) and stores rows directly.
+// instructions of one-K-block stages), issued by two producer warps (A and
+// scales, B) in parallel, and stores rows directly.
 constexpr int kMaskedDecodeTile = 7;
 constexpr int kSplitFixedNs = 1500;  // cluster reduction + pipeline fill of a split CTA
 
@@ -421,11 +422,12 @@ int choose_raster(int num_mb, int rows_per_block, int K)
     return num_mb < want ? (num_mb > 0 ? num_mb : 1) : want;
 }
 
-template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false, int NWG = 2>
+template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false, int NWG = 2,
+          bool PROD2 = false>
 dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_t b_rows,
                           const GemmParams &p, int grid, cudaStream_t stream)
 {
-    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == dg::kKGrouped, NWG>;
+    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == dg::kKGrouped, NWG, PROD2>;
     CUtensorMap ta, tb;
     const bool ok_a = A_MN ? make_tmap_mn(&ta, A, a_rows, static_cast<uint64_t>(p.K), KS * dg::kBK)
                            : make_tmap_operand(&ta, A, static_cast<uint64_t>(p.K), a_rows, dg::kBM, KS);
@@ -457,7 +459,7 @@ dg_status_t launch_kernel(const void *A, uint64_t a_rows, const void *B, uint64_
                             CU_TENSOR_MAP_SWIZZLE_NONE))
             return DG_ERR_CUDA;
     }
-    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT, SPLIT, A_MN, B_MN, NWG>;
+    auto kern = dg::fp8_gemm_kernel<BN, STAGES, KS, LAYOUT, SPLIT, A_MN, B_MN, NWG, PROD2>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices)
@@ -695,8 +697,11 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
     DG_TILE_CASE(128, 5, 1)
     DG_TILE_CASE(224, 2, 2)
     DG_TILE_CASE(256, 3, 1)
-    if constexpr (LAYOUT == dg::kMasked) {
-        DG_TILE_CASE(128, 3, 2)
+    if constexpr (LAYOUT == dg::kMasked && !A_MN && !B_MN) {
+        // decode-sized groups; a second producer warp issues the B boxes
+        if (c.bn == 128 && c.stages == 3 && c.ks == 2 && c.masked_only)
+            return launch_kernel<128, 3, 2, LAYOUT, false, false, false, 2, true>(A, a_rows, B, b_rows, p,
+                                                                                grid, stream);
     }
 #undef DG_TILE_CASE
     if constexpr (LAYOUT == dg::kDense && !B_MN) {
@@ -1276,8 +1281,9 @@ dg_status_t dg_fp8_grouped_gemm_masked(const void *A, const float *sA, const voi
     // Decode-sized groups (at most two 128-row blocks each) make the problem
     // HBM-bound on the weights: the 128-column one-CTA tile with three
     // stages of two K blocks keeps six K blocks in flight per SM with half
-    // the TMA instructions of one-K-block stages, and measured best
-    // (16 x 256 x 4096 x 7168: 156 us, against 172 us for five one-K-block
+    // the TMA instructions of one-K-block stages, its A and B boxes issued by
+    // two producer warps, and measured best (16 x 256 x 4096 x 7168: 144 us,
+    // against 156 us with one producer warp, 172 us for five one-K-block
     // stages and 171-176 us for 112, 224 and 256 columns), unless a tile
     // width or family is pinned.
     if (em <= 2 * dg::kBM && forced_block_n() <= 0 && forced_pair() < 0)

@@ -21,7 +21,9 @@
 //                        section "Hopper TMA特性": TMA for the operands; the
 //                        scales take the LSU path because each TMA
 //                        instruction costs the SM's TMA engine a roughly
-//                        fixed time, whatever its size).
+//                        fixed time, whatever its size).  With PROD2 (the
+//                        masked layout's decode tile) a second warp issues
+//                        the B boxes, in parallel with the A boxes.
 //   warp M (MMA)       : 4 x tcgen05.mma kind::f8f6f4 (K = 32 each) per K
 //                        block into one of NBUF (2..4) TMEM partial buffers,
 //                        issued by one elected lane of a warp-uniform loop
@@ -351,8 +353,14 @@ __device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
 // BN: tile width; STAGES: shared-memory ring depth; KS: 128-wide K blocks per
 // stage (one 3-D TMA box per operand carries all KS blocks -- the TMA engine
 // costs a roughly fixed time per instruction, so bigger boxes move more).
-template <int BN_, int STAGES_, int KS_, bool SPLIT_ = false, bool COLSCALE_ = false, int NWG_ = 2>
+template <int BN_, int STAGES_, int KS_, bool SPLIT_ = false, bool COLSCALE_ = false, int NWG_ = 2,
+          bool PROD2_ = false>
 struct KernelConfig {
+    // PROD2: a second producer warp issues the B boxes while the first
+    // issues the A boxes and the scale copies, so the two TMA instructions
+    // of a stage are issued in parallel (each holds its issuing thread for
+    // a few hundred cycles).
+    static constexpr bool PROD2 = PROD2_;
     // COLSCALE: one B scale per column and K block (the K-grouped layout)
     // instead of one per 128x128 block.
     static constexpr bool COLSCALE = COLSCALE_;
@@ -376,7 +384,8 @@ struct KernelConfig {
     static constexpr int NUM_PROMO_WARPS = 4 * NUM_WG;
     static constexpr int PRODUCER_WARP = NUM_PROMO_WARPS;
     static constexpr int MMA_WARP = NUM_PROMO_WARPS + 1;
-    static constexpr int THREADS = (NUM_PROMO_WARPS + 2) * 32;
+    static constexpr int PRODUCER_B_WARP = NUM_PROMO_WARPS + 2;  // PROD2 only
+    static constexpr int THREADS = (NUM_PROMO_WARPS + 2 + (PROD2_ ? 1 : 0)) * 32;
     static constexpr int A_BYTES = kBM * kBK;  // one K block of A
     static constexpr int B_BYTES = BN * kBK;   // one K block of B
     static constexpr int STAGE_BYTES = KS * (A_BYTES + B_BYTES);
@@ -472,15 +481,18 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float *v)
 // only).  Its stage tile is then loaded as 2-D TMA boxes of 128 M (or N)
 // bytes by 128*KS K rows (B: one box per 128 columns, BN % 128 == 0) and
 // described to the MMA as an MN-major 128-byte-swizzled operand.
-template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false, int NWG = 2>
-__global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped, NWG>::THREADS, 1)
+template <int BN, int STAGES, int KS, int LAYOUT, bool SPLIT, bool A_MN = false, bool B_MN = false, int NWG = 2,
+          bool PROD2 = false>
+__global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped, NWG, PROD2>::THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d64,
                     const __grid_constant__ CUtensorMap tmap_drem, const GemmParams p)
 {
-    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped, NWG>;
+    using Cfg = KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == kKGrouped, NWG, PROD2>;
     static_assert(!SPLIT || LAYOUT == kDense, "K split is implemented for the dense layout");
+    static_assert(!PROD2 || (!SPLIT && !A_MN && !B_MN && LAYOUT != kKGrouped),
+                  "the second producer warp serves K-major persistent tiles");
     static_assert((!A_MN && !B_MN) || LAYOUT == kDense || LAYOUT == kKGrouped,
                   "MN-major operands are implemented for the dense and K-grouped layouts");
     static_assert(LAYOUT != kKGrouped || (A_MN && B_MN), "the K-grouped GEMM is the TN layout");
@@ -522,8 +534,9 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
             tma_prefetch_desc(&tmap_b);
             for (int s = 0; s < STAGES; ++s) {
                 // full: the elected producer lane's expect-tx arrival plus one
-                // cp.async arrival from each of the 32 producer lanes
-                mbar_init(smem_addr(full_bar + s), 1 + 32);
+                // cp.async arrival from each of the 32 producer lanes (and
+                // the B producer's expect-tx arrival)
+                mbar_init(smem_addr(full_bar + s), 1 + 32 + (PROD2 ? 1 : 0));
                 mbar_init(smem_addr(empty_bar + s), 1);
                 mbar_init(smem_addr(sread_bar + s), Cfg::NUM_PROMO_WARPS);
             }
@@ -596,14 +609,16 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
                 }
                 const uint32_t fb = smem_addr(full_bar + stage);
                 if (elect_one()) {
-                    mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
+                    mbar_arrive_expect_tx(fb, PROD2 ? KS * Cfg::A_BYTES : Cfg::STAGE_BYTES);
                     if constexpr (A_MN)
                         tma_load_2d(smem_addr(a_tiles + stage * KS * Cfg::A_BYTES), &tmap_a, fb, a_row,
                                     kb0 * kBK);
                     else
                         tma_load_3d(smem_addr(a_tiles + stage * KS * Cfg::A_BYTES), &tmap_a, fb, 0,
                                     a_row, kb0);
-                    if constexpr (B_MN) {
+                    if constexpr (PROD2) {
+                        // (the B producer warp issues the B box)
+                    } else if constexpr (B_MN) {
                         // [BN/128 column slices][KS*128 K rows][128 bytes]
 #pragma unroll
                         for (int c = 0; c < BN / 128; ++c)
@@ -661,6 +676,43 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
         __syncwarp();
         if constexpr (SPLIT)
             cluster_sync();  // first cluster barrier of the K-split reduction
+    } else if (PROD2 && warp == Cfg::PRODUCER_B_WARP) {
+        // ---------------------------------------------------- B box producer
+        // The same stages as the A producer, one B box each.  On the normal
+        // path the MMA warp waits for every stage, so every box has landed
+        // before the CTA exits; after an abort the boxes in flight get a
+        // bounded moment to land.
+        TileScheduler<LAYOUT, SPLIT> sched(p);
+        TileCoord tc;
+        uint32_t stage = 0, phase = 0;
+        bool ok = !(p.stall_injection && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0);
+        while (ok && sched.next(tc, false)) {
+            const int b_row = tc.g * p.N + tc.nb * BN;
+            const int kb_end = sched.kb_end();
+            for (int kb0 = sched.kb_begin(); kb0 < kb_end; kb0 += KS) {
+                if (!warp_wait_bounded(smem_addr(empty_bar + stage), phase ^ 1, tmo, abort_flag,
+                                       kRoleProducer, 32 + stage)) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
+                    const uint32_t fb = smem_addr(full_bar + stage);
+                    mbar_arrive_expect_tx(fb, KS * Cfg::B_BYTES);
+                    tma_load_3d(smem_addr(b_tiles + stage * KS * Cfg::B_BYTES), &tmap_b, fb, 0, b_row, kb0);
+                }
+                __syncwarp();
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < 200000ull) {
+            }
+        }
+        __syncwarp();
     } else if (warp == Cfg::MMA_WARP) {
         // ------------------------------------------------------- MMA issuer
         // Uniform loop; the descriptors stay warp-uniform and one elected
