@@ -48,10 +48,12 @@ def _run_dense(dg, p):
     (300, 2112, 640),
     (513, 7168, 256),     # wide N: 224/256-column tiles, ragged M tail
     # decode shapes: too few tiles to fill the GPU, so the K range of each
-    # tile is split over a cluster and reduced through distributed shared memory
-    (128, 1024, 4096),
-    (64, 2112, 7168),
-    (100, 4096, 3200),    # 25 K blocks: uneven split
+    # tile is split over a cluster; the splits' fp32 partials meet in an L2
+    # workspace and each CTA sums its rows of them in split order
+    (128, 1024, 4096),    # 8-way split
+    (64, 2112, 7168),     # 8-way split
+    (100, 4096, 3200),    # 25 K blocks: uneven 4-way split
+    (64, 256, 4096),      # 16-way split: 8 rows of each tile per CTA
 ])
 def test_dense_matches_oracle(dg, oracle_mod, M, N, K):
     p = gi.dense_problem(M, N, K, seed_a=1000 + M, seed_b=2000 + N)

@@ -165,6 +165,30 @@ def test_masked_tile_path(dg, oracle_mod, bn):
     assert_close(got[valid], ref[valid], f"masked BN={bn}")
 
 
+def test_masked_decode_tile_path(dg, oracle_mod):
+    """The planner's own tile for decode-sized masked groups (no width or
+    family pinned): 128 columns, three stages of two K blocks, a second
+    producer warp for the B boxes, rows stored directly.  Whole output, with
+    every group's masked rows checked bit for bit; K = 1152 leaves the last
+    stage half outside K, and ragged masked_m values cover partial row
+    blocks, a group of 128 + 1 rows and an empty group."""
+    G, max_m, N, K = 8, 256, N_MID, 1152
+    mm = np.array([1, 129, 256, 0, 64, 200, 128, 17], dtype=np.int32)
+    p = gi.masked_problem(G, max_m, N, K, masked_m=mm, seed_a=520, seed_b=521)
+    plan = _plan(dg, 2, max_m, N, K, G)
+    assert (plan["BN"], plan["stages"], plan["ks"], plan["pair"]) == ("128", "3", "2", "0"), plan
+    A, sA, B, sB, D, m = dev_masked(p)
+    dg.dg_fp8_grouped_gemm_masked(A, sA, B, sB, D, m, 0)
+    st = dg.dg_get_device_status()
+    assert st == 0, dg.dg_status_string(st)
+    got = bits(D)
+    init = np.full((G, max_m, N), SENTINEL, np.uint16)
+    _, ref = oracle_mod.grouped_masked(p["A"], p["sA"], p["B"], p["sB"], p["masked_m"], init)
+    valid = np.arange(max_m)[None, :] < mm[:, None]
+    assert np.array_equal(got[~valid], ref[~valid])
+    assert_close(got[valid], ref[valid], "masked decode tile")
+
+
 @pytest.mark.parametrize("family,layout", [(2, "contiguous"), (1, "masked")])
 def test_grouped_ue8m0_benchmark_tile_path(dg, oracle_mod, family, layout):
     """The UE8M0 tiles the grouped benchmark workloads take: 256 x 224 pairs
