@@ -358,6 +358,12 @@ dg_status_t dg_set_timing_stamps(unsigned long long *stamps);
  * encodes none and leaves this count unchanged. */
 unsigned long long dg_get_tensor_map_encodes(void);
 
+/* Device allocations (cudaMalloc) the library has made so far in this
+ * process: the K-split workspace, allocated on first use per device and
+ * grown when a larger one is needed.  dg_fp8_gemm_nt_noalloc never adds to
+ * it. */
+unsigned long long dg_get_device_allocations(void);
+
 /* Time limit of each pipeline wait inside the kernels, in nanoseconds
  * (default 2e9).  A wait that runs past it makes the kernel record
  * DG_ERR_TIMEOUT, drain its in-flight copies and return.  The output of a

@@ -65,6 +65,7 @@ _SIGNATURES = {
     "dg_set_block_n": (_I, [_I]),
     "dg_set_timing_stamps": (_I, [_P]),
     "dg_get_tensor_map_encodes": (ctypes.c_ulonglong, []),
+    "dg_get_device_allocations": (ctypes.c_ulonglong, []),
     "dg_set_wait_timeout_ns": (_I, [ctypes.c_uint64]),
     "dg_set_stall_injection": (_I, [_I]),
     "dg_get_device_status": (_I, [_P]),
@@ -183,6 +184,11 @@ def dg_set_timing_stamps(stamps) -> None:
 def dg_get_tensor_map_encodes() -> int:
     """Tensor maps encoded so far (cache misses of the library's map cache)."""
     return int(load_library().dg_get_tensor_map_encodes())
+
+
+def dg_get_device_allocations() -> int:
+    """Device allocations (cudaMalloc) the library has made so far."""
+    return int(load_library().dg_get_device_allocations())
 
 
 def dg_set_wait_timeout_ns(ns: int) -> None:

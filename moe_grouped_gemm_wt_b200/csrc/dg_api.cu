@@ -215,6 +215,7 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 std::mutex g_ws_mutex;
 void *g_ws_ptr[kMaxDevices] = {};
 size_t g_ws_bytes[kMaxDevices] = {};
+std::atomic<uint64_t> g_device_allocs{0};  // cudaMalloc calls made (dg_get_device_allocations)
 
 dg_status_t split_workspace(int dev, size_t bytes, void **out)
 {
@@ -229,6 +230,7 @@ dg_status_t split_workspace(int dev, size_t bytes, void **out)
             g_ws_bytes[dev] = 0;
         }
         void *ptr = nullptr;
+        g_device_allocs.fetch_add(1);
         if (cudaMalloc(&ptr, bytes) != cudaSuccess) {
             (void)cudaGetLastError();
             return DG_ERR_CUDA;
@@ -1452,6 +1454,8 @@ dg_status_t dg_set_block_n(int n)
 }
 
 unsigned long long dg_get_tensor_map_encodes(void) { return g_tmap_encodes.load(); }
+
+unsigned long long dg_get_device_allocations(void) { return g_device_allocs.load(); }
 
 dg_status_t dg_set_timing_stamps(unsigned long long *stamps)
 {
