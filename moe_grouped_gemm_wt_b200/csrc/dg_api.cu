@@ -884,6 +884,15 @@ dg_status_t launch_bs(const void *A, uint64_t a_rows, const void *B, uint64_t b_
     } else {
         tdrem = td64;
     }
+    if (SPLIT && p.ksplit >= 2 && dg::kBM % p.ksplit == 0) {
+        // the K-split reduction's maps: the partials and one CTA's output rows
+        const int rows_per = dg::kBM / p.ksplit;
+        const uint64_t tiles = static_cast<uint64_t>(p.num_mb) * static_cast<uint64_t>(p.num_nb);
+        if (!make_tmap_split_ws(&td64, p.ws, BN, p.ksplit, tiles, rows_per) ||
+            !make_tmap_bf16(&tdrem, p.D, static_cast<uint64_t>(p.N), a_rows, BN, rows_per,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+            return DG_ERR_CUDA;
+    }
     auto kern = dg::fp8_gemm_bs_kernel<BN, STAGES, KS, LAYOUT, PAIR, SPLIT>;
     static std::atomic<bool> attr_set[kMaxDevices];
     const int dev = current_device();

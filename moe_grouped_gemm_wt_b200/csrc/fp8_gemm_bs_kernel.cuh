@@ -130,7 +130,13 @@ struct BsConfig {
     static constexpr int SF_SLOT_COLS = 16;
     static constexpr int TSLOTS = (512 - SF_COL0) / SF_SLOT_COLS >= 4 ? 4 : (512 - SF_COL0) / SF_SLOT_COLS;
     static constexpr int TMEM_COLS = SF_COL0 + TSLOTS * SF_SLOT_COLS <= 256 ? 256 : 512;
-    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * NACC + 2 * SF_RING + 2 * TSLOTS) + 16;
+    // (+ one barrier for the K-split reduction's TMA load)
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * NACC + 2 * SF_RING + 2 * TSLOTS + 1) + 16;
+    // K split: the reduction reads this CTA's rows of all S partials
+    // (BN/4 x 128 float4s whatever S is) into the idle operand ring at
+    // offset 0, and stages its bf16 rows (at most 64 x BN) after them.
+    static constexpr int RED_IN_BYTES = (BN / 4) * kBM * 16;
+    static constexpr int RED_OUT_OFFSET = (RED_IN_BYTES + 1023) / 1024 * 1024;
     static constexpr int EPI_FULL_BOXES = BN / 64;
     static constexpr int EPI_REM = BN % 64;
     static constexpr int EPI_BOXES = EPI_FULL_BOXES + (EPI_REM > 0 ? 1 : 0);
@@ -150,6 +156,8 @@ struct BsConfig {
     static_assert(4 + 4 * SFB_CHUNKS <= SF_SLOT_COLS, "scale slot too small");
     static_assert(B_BYTES % 1024 == 0, "B tiles must keep 1024-byte swizzle atoms aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+    static_assert(!SPLIT || RED_OUT_OFFSET + 64 * BN * 2 <= STAGES * (STAGE_A + STAGE_B),
+                  "the split reduction's buffers fit in the operand ring");
 };
 
 template <int BN, int STAGES, int KS, int LAYOUT, bool PAIR, bool SPLIT = false>
@@ -184,7 +192,8 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
     uint64_t *staged_empty = staged_full + Cfg::SF_RING;  // scale writers are done with the slot
     uint64_t *sf_full = staged_empty + Cfg::SF_RING;      // (leader) TMEM scale slot written by every CTA
     uint64_t *sf_empty = sf_full + TSLOTS;                // MMAs reading the scale slot done
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sf_empty + TSLOTS);
+    uint64_t *red_bar = sf_empty + TSLOTS;                 // K split: the reduction's partials landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(red_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     uint8_t *epi_stage = smem + Cfg::EPI_OFFSET;
 
@@ -211,13 +220,16 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
             mbar_init(smem_addr(sf_full + t), CTAS * 4);
             mbar_init(smem_addr(sf_empty + t), 1);
         }
+        mbar_init(smem_addr(red_bar), 1);
         *abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmap_a);
         tma_prefetch_desc(&tmap_b);
-        if (Cfg::EPI_FULL_BOXES > 0)
+        // (K split: tmap_d64 describes the partials, tmap_drem the
+        // reduction's output rows)
+        if (SPLIT || Cfg::EPI_FULL_BOXES > 0)
             tma_prefetch_desc(&tmap_d64);
-        if (Cfg::EPI_REM > 0)
+        if (SPLIT || Cfg::EPI_REM > 0)
             tma_prefetch_desc(&tmap_drem);
     }
     if (warp == Cfg::MMA_WARP) {
@@ -652,6 +664,56 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
             constexpr int C4 = BN / 4;
             const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
             const float4 *src0 = reinterpret_cast<const float4 *>(p.ws) + tile * S * C4 * kBM;
+            if (kBM % S == 0) {
+                // One TMA box brings this CTA's rows of all S partials,
+                // [S][C4][rows_per] float4s, into the idle operand ring; the
+                // sums (in split order) are rounded, staged as
+                // [rows_per][BN] bf16 and stored with one TMA box (rows past
+                // M and columns past N are clipped).
+                const float4 *red_in = reinterpret_cast<const float4 *>(smem);
+                uint8_t *red_out = smem + Cfg::RED_OUT_OFFSET;
+                const int r0 = static_cast<int>(rank_s) * rows_per;
+                if (threadIdx.x == 0) {
+                    // the partials were written by generic-proxy stores
+                    fence_proxy_async_global();
+                    mbar_arrive_expect_tx(smem_addr(red_bar), Cfg::RED_IN_BYTES);
+                    tma_load_4d(smem_addr(smem), &tmap_d64, smem_addr(red_bar), 4 * r0, 0, 0,
+                                static_cast<int>(tile));
+                }
+                // the box must land whatever the abort flag says: this CTA's
+                // shared memory may not be left while the copy is in flight
+                int got_lane = 0;
+                if (lane == 0)
+                    got_lane = wait_bounded(smem_addr(red_bar), 0, drain_tmo, abort_flag, kRoleDrain, 40, false)
+                                   ? 1 : 0;
+                const bool got = __shfl_sync(0xFFFFFFFFu, got_lane, 0) != 0;
+                if (got) {
+                    for (int it = threadIdx.x; it < rows_per * C4; it += Cfg::THREADS) {
+                        const int lr = it % rows_per;  // rows fastest: conflict-free reads
+                        const int c4 = it / rows_per;
+                        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int src = 0; src < S; ++src) {
+                            const float4 v = red_in[(src * C4 + c4) * rows_per + lr];
+                            sum.x += v.x;
+                            sum.y += v.y;
+                            sum.z += v.z;
+                            sum.w += v.w;
+                        }
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(sum.x, sum.y);
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(sum.z, sum.w);
+                        uint2 u;
+                        u.x = *reinterpret_cast<uint32_t *>(&h0);
+                        u.y = *reinterpret_cast<uint32_t *>(&h1);
+                        *reinterpret_cast<uint2 *>(red_out + (lr * BN + 4 * c4) * 2) = u;
+                    }
+                }
+                fence_proxy_async_smem();
+                if (__syncthreads_and(got ? 1 : 0) && threadIdx.x == 0) {
+                    tma_store_2d(&tmap_drem, smem_addr(red_out), tc.nb * BN, tc.mb * kBM + r0);
+                    bulk_commit_group();
+                    bulk_wait_group<0>();
+                }
+            } else
             for (int it = threadIdx.x; it < rows_per * C4; it += Cfg::THREADS) {
                 const int lr = it % rows_per;  // rows fastest: contiguous reads
                 const int c4 = it / rows_per;
