@@ -170,6 +170,28 @@ def test_ue8m0_planner_under_an_sm_cap(lib):
         lib.dg_set_num_sms(0)
 
 
+def test_masked_decode_tile_choice(lib):
+    """The fp32-scale masked planner (host only): decode-sized groups (max_m
+    at most two 128-row blocks) take the 128-column tile of three two-K-block
+    stages; larger groups go through the general cost model; a pinned tile
+    width is honoured."""
+    buf = ctypes.create_string_buffer(256)
+    desc = lambda *a: (lib.dg_describe_config(*a, buf, 256), dict(kv.split("=") for kv in buf.value.decode().split()))[1]
+    assert lib.dg_set_num_sms(148) == 0
+    try:
+        for max_m in (1, 128, 200, 256):
+            d = desc(2, max_m, 4096, 7168, 16)
+            assert (d["BN"], d["stages"], d["ks"], d["pair"]) == ("128", "3", "2", "0"), (max_m, d)
+        d = desc(2, 1024, 4096, 7168, 16)
+        assert (d["stages"], d["ks"]) != ("3", "2") or d["BN"] != "128", d
+        assert lib.dg_set_block_n(256) == 0
+        d = desc(2, 256, 4096, 7168, 16)
+        assert d["BN"] == "256", d
+    finally:
+        lib.dg_set_block_n(0)
+        lib.dg_set_num_sms(0)
+
+
 def test_noalloc_split_choice_under_an_sm_cap(lib):
     """The split count of dg_fp8_gemm_nt_noalloc (host only, dg_describe_config
     layout 6): every split gets the same number (at least two) of K blocks,
