@@ -664,7 +664,8 @@ __global__ void __launch_bounds__(BsConfig<BN, STAGES, KS, PAIR, SPLIT>::THREADS
             constexpr int C4 = BN / 4;
             const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
             const float4 *src0 = reinterpret_cast<const float4 *>(p.ws) + tile * S * C4 * kBM;
-            if (kBM % S == 0) {
+            if (S >= 2 && kBM % S == 0) {
+                // (the same condition under which the host built the two maps)
                 // One TMA box brings this CTA's rows of all S partials,
                 // [S][C4][rows_per] float4s, into the idle operand ring; the
                 // sums (in split order) are rounded, staged as

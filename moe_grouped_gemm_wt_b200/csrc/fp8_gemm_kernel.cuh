@@ -1062,7 +1062,8 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
             constexpr int C4 = BN / 4;
             const size_t tile = static_cast<size_t>(tc.mb) * p.num_nb + tc.nb;
             const float4 *src0 = reinterpret_cast<const float4 *>(p.ws) + tile * S * C4 * kBM;
-            if (p.D32 == nullptr && kBM % S == 0) {
+            if (p.D32 == nullptr && S >= 2 && kBM % S == 0) {
+                // (the same condition under which the host built the two maps)
                 // bf16 output.  One TMA box brings this CTA's rows of all S
                 // partials, [S][C4][rows_per] float4s, into the idle operand
                 // ring; the sums (in split order, as below) are rounded,

@@ -46,6 +46,7 @@ def dg():
     (64, 1024, 2048),
     (300, 2112, 1152),   # three row blocks, 9 K blocks (split 2 ways: 5 + 4)
     (1024, 2112, 896),   # 120 tiles: the scratch bounds the split
+    (2048, 2112, 1152),  # 240 tiles: only an unsplit pass (S = 1) fits the scratch
 ])
 def test_noalloc_matches_oracle_and_default_entry_point(dg, oracle_mod, M, N, K):
     p = gi.dense_problem(M, N, K, seed_a=300 + M, seed_b=400 + N)
