@@ -23,7 +23,8 @@ this method) on the same workload and metric, rank 0 only.
 (inputs quantised with power-of-two scales, packed four to an int32; the
 tensor core applies them).  The default run also reports that mode's
 per-shape numbers under "ue8m0_shapes"; the headline stays the fp32-scale
-mode.
+mode.  It also times the NN, TN and TT operand layouts of the dense GEMM on
+the decode and prefill shapes ("layout_shapes").
 """
 from __future__ import annotations
 
@@ -196,7 +197,9 @@ def pack_ue8m0(dg, p, d):
 
 def to_device(p, torch, dev, dg=None):
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-    out = dict(A=t(p["A"]), B=t(p["B"]), sA=t(gi.sa_to_kernel_layout(p["sA"])), sB=t(p["sB"]))
+    a_mn, b_mn = OPERAND_LAYOUTS.get(p.get("layout"), (False, False))
+    out = dict(A=t(p["A"].T if a_mn else p["A"]), B=t(p["B"].T if b_mn else p["B"]),
+               sA=t(gi.sa_to_kernel_layout(p["sA"])), sB=t(p["sB"]))
     if p["kind"] == "dense":
         out["D"] = torch.empty((p["M"], p["N"]), dtype=torch.bfloat16, device=dev)
     elif p["kind"] == "contiguous":
@@ -221,7 +224,9 @@ def call(dg, p, d, stream=None):
             dg.dg_fp8_grouped_gemm_masked_ue8m0(d["A"], d["sfa"], d["B"], d["sfb"], d["D"], d["masked_m"],
                                                 expected_m=int(np.mean(p["masked_m"])), stream=stream)
         return
-    if p["kind"] == "dense":
+    if p.get("layout"):
+        getattr(dg, "dg_fp8_gemm_" + p["layout"])(d["A"], d["sA"], d["B"], d["sB"], d["D"], stream=stream)
+    elif p["kind"] == "dense":
         dg.dg_fp8_gemm_nt(d["A"], d["sA"], d["B"], d["sB"], d["D"], stream=stream)
     elif p["kind"] == "contiguous":
         dg.dg_fp8_grouped_gemm_contiguous(d["A"], d["sA"], d["B"], d["sB"], d["D"], d["m_indices"],
@@ -284,8 +289,15 @@ def workload_label(p, name):
     return f"{name} G={p['G']} max_m={p['max_m']} N={p['N']} K={p['K']} sum_masked_m={int(p['masked_m'].sum())}"
 
 
+# Operand layouts of the dense GEMM besides NT: (A stored M-major, B stored
+# N-major) for the layout entry points dg_fp8_gemm_nn / _tn / _tt.
+OPERAND_LAYOUTS = {"nn": (False, True), "tn": (True, True), "tt": (True, False)}
+
+
 def tile_label(dg, p):
     base = 3 if p.get("ue8m0") else 0  # describe_config layouts 3-5: the UE8M0 mode
+    if p.get("layout"):
+        return f"operand layout {p['layout']} (one-CTA tiles, MN-major boxes)"
     if p["kind"] == "dense":
         return dg.dg_describe_config(base, p["M"], p["N"], p["K"], 1)
     if p["kind"] == "contiguous":
@@ -532,11 +544,35 @@ def run_ours(args):
                 torch.cuda.empty_cache()
         return out
 
-    shapes, ue8m0_shapes = {}, None
+    # the NN / TN / TT operand layouts on the two dense shapes (fp32 scales)
+    def sweep_layouts():
+        out = {}
+        for name in ("dense_decode", "dense_prefill"):
+            for lay in sorted(OPERAND_LAYOUTS):
+                q = make_problem(name, False)
+                q["layout"] = lay
+                dq = to_device(q, torch, dev, dg)
+                kq = []
+                tq = time_kernel(torch, dg, q, dq, max(10, min(args.steps, 30)), 3, flush, kq)
+                mq, kmq = statistics.median(tq), statistics.median(kq)
+                fq, bq, _ = workload_cost(q)
+                bound, t_roof, _ = roofline(fq, bq, pk)
+                out[f"{name}:{lay}"] = {
+                    "us": mq * 1e3, "tflops": fq / (mq * 1e-3) / 1e12, "bound": bound,
+                    "frac_of_roofline": t_roof / (mq * 1e-3), "kernel_us": kmq * 1e3,
+                    "kernel_frac_of_roofline": t_roof / (kmq * 1e-3), "tile": tile_label(dg, q),
+                }
+                del dq
+                torch.cuda.empty_cache()
+        return out
+
+    shapes, ue8m0_shapes, layout_shapes = {}, None, None
     if not args.no_shapes:
         shapes = sweep(ue8m0)
         if not ue8m0 and not args.no_ue8m0_shapes:
             ue8m0_shapes = sweep(True)
+        if not ue8m0 and not args.no_layout_shapes:
+            layout_shapes = sweep_layouts()
     clocks = sampler.stop()
 
     e2e_ms, h2d, d2h = time_e2e(torch, dg, p, max(10, min(args.steps, 50)), 3, dev)
@@ -600,6 +636,8 @@ def run_ours(args):
     }
     if ue8m0_shapes is not None:
         line["ue8m0_shapes"] = ue8m0_shapes
+    if layout_shapes is not None:
+        line["layout_shapes"] = layout_shapes
     print(json.dumps(line), flush=True)
     return 0
 
@@ -615,6 +653,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--scales", choices=("fp32", "ue8m0"), default="fp32",
                     help="fp32 scales (the headline mode) or the UE8M0 block-scaled mode")
+    ap.add_argument("--no-layout-shapes", action="store_true",
+                    help="skip the NN / TN / TT operand-layout timings of the dense shapes")
     ap.add_argument("--no-ue8m0-shapes", action="store_true",
                     help="skip the UE8M0 mode's per-shape sweep of a default run")
     ap.add_argument("--workload", choices=sorted(gi.WORKLOADS), default=HEADLINE,
