@@ -108,7 +108,9 @@ dg_status_t dg_fp8_gemm_nt(const void *A, const float *sA, const void *B,
  * sA, sB and D are as in dg_fp8_gemm_nt (sA [K/128][M_pad], sB
  * [ceil(N/128)][K/128], D [M][N] bf16).  An M-major A needs M % 16 == 0
  * (DG_ERR_UNSUPPORTED otherwise).  These layouts run on one-CTA tiles; an
- * N-major B uses 128- or 256-column tiles and no K split.
+ * N-major B uses 128- or 256-column tiles (whole 128-column boxes), and a
+ * decode-shaped problem splits its K range over a cluster on 128-column
+ * tiles (the library-owned split workspace of dg_fp8_gemm_nt, same rules).
  */
 dg_status_t dg_fp8_gemm_nn(const void *A, const float *sA, const void *B,
                            const float *sB, void *D, int M, int N, int K,

@@ -257,11 +257,12 @@ struct TileChoice {
     int wg = 2;      // promotion warpgroups
     int rebal = 0;   // pair tiles: registers rebalanced with setmaxnreg (always for wg >= 3)
     int masked_only = 0;  // taken only by the masked layout's decode-sized groups
+    int nmajor_split = 0;  // the K split of an N-major B (whole 128-column boxes) only
 };
 constexpr TileChoice kTileChoices[] = {
     {112, 3, 2, 0, 0.41, 0, 1.9}, {128, 5, 1, 0, 0.53, 0, 1.9}, {224, 2, 2, 0, 0.78, 0, 1.9},
     {256, 3, 1, 0, 0.68, 0, 1.9}, {144, 3, 2, 1, 0.40, 0, 1.9, 3}, {160, 3, 2, 0, 0.441, 1, 2.2},
-    {192, 3, 2, 0, 0.50, 1, 2.2, 3}, {128, 3, 2, 0, 0.50, 0, 1.9, 2, 0, 1},
+    {192, 3, 2, 0, 0.50, 1, 2.2, 3}, {128, 3, 2, 0, 0.50, 0, 1.9, 2, 0, 1}, {128, 3, 2, 1, 0.40, 0, 1.9, 2, 0, 0, 1},
 };
 // The masked layout's tile for decode-sized groups (at most two 128-row
 // blocks per group): HBM-bound on the weights, it keeps six K blocks in
@@ -339,7 +340,7 @@ Plan choose_plan(int64_t m_blocks, int64_t pair_rows, int N, int num_kb, int sms
     Plan best{kTileChoices[0], 1};
     double best_cost = 1e300;
     if (limits & kWholeBoxes) {
-        allow_split = false;
+        // (an N-major B splits K only on the 128-column split tile)
         for (const TileChoice &c : kTileChoices)
             if (!c.pair && !c.split && c.bn % 128 == 0) {
                 best = Plan{c, 1};
@@ -357,6 +358,8 @@ Plan choose_plan(int64_t m_blocks, int64_t pair_rows, int N, int num_kb, int sms
         if (forced_pair() >= 0 && c.pair != forced_pair())
             continue;
         if (c.masked_only)
+            continue;
+        if (c.nmajor_split != ((limits & kWholeBoxes) != 0 && c.split))
             continue;
         if (c.pair) {
             const int pairs = sms / 2;
@@ -616,7 +619,10 @@ int query_max_clusters(int S)
 int max_active_clusters(const TileChoice &c, int S)
 {
     static int cache[kMaxDevices][5] = {};  // S = 2, 4, 8, 16 (index log2(S))
-    if (c.bn != 144 || S < 1)
+    // The 128-column split tile of an N-major B uses a little less shared
+    // memory than the 144-column one and runs one CTA per SM too: the same
+    // clusters fit.
+    if ((c.bn != 144 && c.bn != 128) || !c.split || S < 1)
         return 0;
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) {
@@ -710,6 +716,12 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
         if (c.bn == 144 && c.stages == 3 && c.ks == 2 && c.split && c.wg == 3)
             return launch_kernel<144, 3, 2, LAYOUT, true, A_MN, false, 3>(A, a_rows, B, b_rows, p, grid,
                                                                           stream);
+    }
+    if constexpr (LAYOUT == dg::kDense && B_MN) {
+        // an N-major B splits K on whole 128-column boxes
+        if (c.bn == 128 && c.stages == 3 && c.ks == 2 && c.split && c.nmajor_split)
+            return launch_kernel<128, 3, 2, LAYOUT, true, A_MN, true, 2>(A, a_rows, B, b_rows, p, grid,
+                                                                         stream);
     }
     return DG_ERR_UNSUPPORTED;
 }
