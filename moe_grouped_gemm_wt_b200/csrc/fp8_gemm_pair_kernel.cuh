@@ -336,8 +336,14 @@ __global__ void __launch_bounds__(PairConfig<BN, STAGES, KS, NWG, REBAL>::THREAD
                     if (is_a) {
                         if (leader)
                             mbar_arrive_expect_tx(smem_addr(full_bar + stage), 2 * KS * Cfg::A_BYTES);
-                        tma_load_3d_pair(smem_addr(a_tiles + stage * KS * Cfg::A_BYTES), &tmap_a, fb, 0,
-                                         a_row, kb0);
+                        // dense: A rows are read again by the band's other
+                        // column tiles while B streams past -- keep them in L2
+                        if (LAYOUT == kDense)
+                            tma_load_3d_pair_hint(smem_addr(a_tiles + stage * KS * Cfg::A_BYTES), &tmap_a, fb,
+                                                  0, a_row, kb0, l2_policy_evict_last());
+                        else
+                            tma_load_3d_pair(smem_addr(a_tiles + stage * KS * Cfg::A_BYTES), &tmap_a, fb, 0,
+                                             a_row, kb0);
                     } else {
                         if (leader)
                             mbar_arrive_expect_tx(smem_addr(full_bar + stage), 2 * KS * Cfg::B_BYTES);

@@ -208,6 +208,25 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void *tmap,
         : "memory");
 }
 
+// An L2 cache policy that keeps lines in L2 in preference to others (for
+// operands that later tiles read again while other operands stream past).
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+// tma_load_3d_pair with an L2 cache policy for the loaded lines.
+__device__ __forceinline__ void tma_load_3d_pair_hint(uint32_t dst, const void *tmap, uint32_t bar_cluster, int x,
+                                                      int y, int z, uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z), "l"(pol)
+        : "memory");
+}
+
 // 2-D tiled store of a shared-memory box to global memory (bulk group).
 // Elements outside the tensor's extent are not written.
 __device__ __forceinline__ void tma_store_2d(const void *tmap, uint32_t src, int x, int y)
