@@ -245,7 +245,10 @@ dg_status_t split_workspace(int dev, size_t bytes, void **out)
 // ---------------------------------------------------------- configurations
 
 // The tile widths compiled into the library.  Each has a pipeline depth that
-// fills the 227 KB of shared memory (one CTA per SM).
+// fills the 227 KB of shared memory (one CTA per SM).  128x256 comes twice:
+// three stages with whole-tile staged TMA stores (cheaper per tile: short K
+// ranges) and four stages with per-warp stores (cheaper per K block: long K
+// ranges); the cost model picks between them.
 struct TileChoice {
     int bn;
     int stages;
@@ -263,6 +266,7 @@ constexpr TileChoice kTileChoices[] = {
     {112, 3, 2, 0, 0.41, 0, 1.9}, {128, 5, 1, 0, 0.53, 0, 1.9}, {224, 2, 2, 0, 0.78, 0, 1.9},
     {256, 3, 1, 0, 0.68, 0, 1.9}, {144, 3, 2, 1, 0.40, 0, 1.9, 3}, {160, 3, 2, 0, 0.441, 1, 2.2},
     {192, 3, 2, 0, 0.50, 1, 2.2, 3}, {128, 3, 2, 0, 0.50, 0, 1.9, 2, 0, 1}, {128, 3, 2, 1, 0.40, 0, 1.9, 2, 0, 0, 1},
+    {256, 4, 1, 0, 0.655, 0, 2.6},
 };
 // The masked layout's tile for decode-sized groups (at most two 128-row
 // blocks per group): HBM-bound on the weights, it keeps six K blocks in
@@ -705,6 +709,7 @@ dg_status_t dispatch(const Plan &plan, const void *A, uint64_t a_rows, const voi
     DG_TILE_CASE(128, 5, 1)
     DG_TILE_CASE(224, 2, 2)
     DG_TILE_CASE(256, 3, 1)
+    DG_TILE_CASE(256, 4, 1)
     if constexpr (LAYOUT == dg::kMasked && !A_MN && !B_MN) {
         // decode-sized groups; a second producer warp issues the B boxes
         if (c.bn == 128 && c.stages == 3 && c.ks == 2 && c.masked_only)

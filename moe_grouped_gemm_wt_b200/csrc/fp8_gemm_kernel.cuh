@@ -415,14 +415,19 @@ struct KernelConfig {
     // One staging buffer per output box when shared memory allows, so a
     // warpgroup stores all its boxes without waiting for an earlier store to
     // finish reading its buffer; else one buffer reused box after box.  A
-    // ring too deep for even one buffer per warpgroup (the masked decode
-    // tile) stores every row segment directly (EPI_STAGED false).
+    // ring too deep for even one buffer per warpgroup (EPI_STAGED false)
+    // leaves room only for a small buffer per promotion warp (below).
     static constexpr int EPI_BOXES = EPI_FULL_BOXES + (EPI_REM > 0 ? 1 : 0);
     static constexpr bool EPI_STAGED = 1024 + EPI_OFFSET + NUM_WG * EPI_WG_BYTES <= 232448;
     static constexpr int EPI_BUFS =
         1024 + EPI_OFFSET + NUM_WG * EPI_BOXES * EPI_WG_BYTES <= 232448 ? EPI_BOXES : 1;
+    // Without whole-tile staging, each promotion warp stages 32 rows x 32
+    // columns of bf16 at a time and writes them back with row-contiguous
+    // stores.
+    static constexpr int EPI_WARP_BYTES = 32 * 32 * 2;
     static constexpr int SMEM_BYTES =
-        1024 /*align slack*/ + EPI_OFFSET + ((SPLIT || !EPI_STAGED) ? 0 : NUM_WG * EPI_BUFS * EPI_WG_BYTES);
+        1024 /*align slack*/ + EPI_OFFSET +
+        (SPLIT ? 0 : EPI_STAGED ? NUM_WG * EPI_BUFS * EPI_WG_BYTES : NUM_PROMO_WARPS * EPI_WARP_BYTES);
 
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128: multiple of 16, <= 256");
     static_assert(BN % NUM_WG == 0 && BN_WG % 4 == 0, "promotion columns per warpgroup: a multiple of 4");
@@ -435,6 +440,7 @@ struct KernelConfig {
     static_assert(KS >= 1 && KS <= 4, "K blocks per stage");
     static_assert(EPI_REM % 8 == 0, "remainder box must be whole 16-byte chunks");
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+    static_assert(SPLIT || EPI_STAGED || BN_WG % 32 == 0, "per-warp epilogue rounds of 32 columns");
     static_assert(!SPLIT || BN_WG % 4 == 0, "split reduction works on float4 columns");
     static_assert(!SPLIT || RED_OUT_OFFSET + 64 * BN * 2 <= STAGES * STAGE_BYTES,
                   "the split reduction's buffers fit in the operand ring");
@@ -1025,14 +1031,45 @@ __global__ void __launch_bounds__(KernelConfig<BN, STAGES, KS, SPLIT, LAYOUT == 
                         bulk_commit_group();
                     }
                 }
-            } else if (row_ok) {
-                const size_t grow = (LAYOUT == kMasked ? static_cast<size_t>(tc.g) * p.M : 0) +
-                                    static_cast<size_t>(m_local);
-                __nv_bfloat16 *drow = p.D + grow * p.N + col0;
+            } else if constexpr (Cfg::EPI_STAGED) {
+                if (row_ok) {
+                    const size_t grow = (LAYOUT == kMasked ? static_cast<size_t>(tc.g) * p.M : 0) +
+                                        static_cast<size_t>(m_local);
+                    __nv_bfloat16 *drow = p.D + grow * p.N + col0;
 #pragma unroll
-                for (int c = 0; c < BN_WG; c += 8)
-                    if (col0 + c < p.N)
-                        *reinterpret_cast<uint4 *>(drow + c) = pack_bf16x8(acc + c);
+                    for (int c = 0; c < BN_WG; c += 8)
+                        if (col0 + c < p.N)
+                            *reinterpret_cast<uint4 *>(drow + c) = pack_bf16x8(acc + c);
+                }
+            } else {
+                // Each warp puts 32 rows x 32 columns of bf16 into its own
+                // 2 KB buffer (16-byte chunk c of row r at slot c ^ ((r/2) % 4):
+                // conflict-free both ways) and reads them back so that four
+                // lanes cover one row's 64 bytes: every store instruction
+                // writes 8 row segments.  Rows that may not be written are
+                // skipped by the lanes that hold them.
+                const uint32_t wbuf = smem_addr(epi_stage) + static_cast<uint32_t>(warp * Cfg::EPI_WARP_BYTES);
+                const unsigned rows = __ballot_sync(0xFFFFFFFFu, row_ok);
+                const size_t grow0 = (LAYOUT == kMasked ? static_cast<size_t>(tc.g) * p.M : 0) +
+                                     static_cast<size_t>(tc.mb) * kBM + static_cast<size_t>(quad * 32);
+#pragma unroll
+                for (int cb = 0; cb < BN_WG; cb += 32) {
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+                        st_shared_v4(wbuf + lane * 64 + ((ch ^ ((lane >> 1) & 3)) * 16),
+                                     pack_bf16x8(acc + cb + ch * 8));
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int r = 8 * j + lane / 4;
+                        const int ch = lane % 4;
+                        const uint4 v = ld_shared_v4u(wbuf + r * 64 + ((ch ^ ((r >> 1) & 3)) * 16));
+                        const int gcol = col0 + cb + ch * 8;
+                        if (((rows >> r) & 1u) != 0u && gcol < p.N)
+                            *reinterpret_cast<uint4 *>(p.D + (grow0 + r) * p.N + gcol) = v;
+                    }
+                    __syncwarp();
+                }
             }
         }
         if constexpr (SPLIT) {

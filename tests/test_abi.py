@@ -192,6 +192,28 @@ def test_masked_decode_tile_choice(lib):
         lib.dg_set_num_sms(0)
 
 
+def test_two_depths_of_the_256_column_tile(lib):
+    """The fp32-scale planner (host only) with the tile width pinned to 256
+    and one-CTA tiles: a short K range (16 K blocks, the contiguous MoE
+    shape) takes three stages with staged TMA stores, a long one (56 or 144
+    K blocks) four stages with per-warp stores."""
+    buf = ctypes.create_string_buffer(256)
+    desc = lambda *a: (lib.dg_describe_config(*a, buf, 256), dict(kv.split("=") for kv in buf.value.decode().split()))[1]
+    assert lib.dg_set_num_sms(148) == 0
+    try:
+        assert lib.dg_set_block_n(256) == 0
+        assert lib.dg_set_tile_family(1) == 0
+        d = desc(1, 32768, 7168, 2048, 8)
+        assert (d["BN"], d["stages"], d["ks"], d["pair"]) == ("256", "3", "1", "0"), d
+        for K in (7168, 18432):
+            d = desc(0, 4096, 7168, K, 1)
+            assert (d["BN"], d["stages"], d["ks"], d["pair"]) == ("256", "4", "1", "0"), (K, d)
+    finally:
+        lib.dg_set_block_n(0)
+        lib.dg_set_tile_family(0)
+        lib.dg_set_num_sms(0)
+
+
 def test_noalloc_split_choice_under_an_sm_cap(lib):
     """The split count of dg_fp8_gemm_nt_noalloc (host only, dg_describe_config
     layout 6): every split gets the same number (at least two) of K blocks,

@@ -6,7 +6,8 @@ the full GPU (several waves of tiles, no SM cap) with ragged M and N (partial
 last row block and partial last column tile) and an odd number of K blocks
 (a two-block pipeline stage with one block past K).  dg_set_block_n and
 dg_set_tile_family force each path, and dg_describe_config confirms it:
-  * fp32-scale one-CTA tiles of 112, 128, 224 and 256 columns,
+  * fp32-scale one-CTA tiles of 112, 128, 224 and 256 columns (the 256-column
+    tile in both depths: three stages on a short K range, four on a long one),
   * fp32-scale CTA-pair tiles of 160 and 192 columns,
   * the K-split decode tile (144 columns over a cluster),
   * the UE8M0 mode's one-CTA and pair tiles of 128, 160, 192 and 224 columns,
@@ -77,6 +78,24 @@ def test_dense_fp32_tile_path(dg, dense_mid, bn, family):
         st = dg.dg_get_device_status()
     assert st == 0, dg.dg_status_string(st)
     assert_close(bits(D), ref, f"dense BN={bn} family={family}")
+
+
+def test_dense_fp32_four_stage_tile(dg, oracle_mod):
+    """128x256 tiles over a long K range (40 K blocks) take the four-stage
+    ring, whose output goes through per-warp staging buffers; ragged M and N,
+    several row blocks and column tiles, whole output against the oracle."""
+    M, N, K = 600, 1040, 5120
+    p = gi.dense_problem(M, N, K, seed_a=511, seed_b=512)
+    _, ref = oracle_mod.gemm_nt(p["A"], p["sA"], p["B"], p["sB"], want_f64=False)
+    with forced(dg, 256, 1):
+        assert _plan(dg, 0, M_MID, N_MID, K_MID)["stages"] == "3"
+        plan = _plan(dg, 0, M, N, K)
+        assert (plan["BN"], plan["stages"], plan["ks"], plan["pair"], plan["ksplit"]) == ("256", "4", "1", "0", "1"), plan
+        A, sA, B, sB, D = dev_dense(p)
+        dg.dg_fp8_gemm_nt(A, sA, B, sB, D)
+        st = dg.dg_get_device_status()
+    assert st == 0, dg.dg_status_string(st)
+    assert_close(bits(D), ref, "dense BN=256 four stages")
 
 
 def test_dense_k_split_path(dg, oracle_mod):
