@@ -184,10 +184,46 @@ def test_masked_tile_path(dg, oracle_mod, bn):
     assert_close(got[valid], ref[valid], f"masked BN={bn}")
 
 
+
+def test_grouped_four_stage_tile(dg, oracle_mod):
+    """The four-stage 128x256 tile (a long K range, 40 K blocks) in both
+    grouped layouts: its per-warp staged stores must leave every padding row
+    of the contiguous layout and every masked row untouched, bit for bit,
+    while partial row blocks and a ragged last column tile are written."""
+    N, K = 1040, 5120
+    pc = gi.contiguous_problem([300, 0, 517, 128], N, K, seed_a=530, seed_b=531)
+    G, max_m = 4, 384
+    mm = np.array([384, 1, 0, 250], dtype=np.int32)
+    pm = gi.masked_problem(G, max_m, N, K, masked_m=mm, seed_a=532, seed_b=533)
+    with forced(dg, 256, 1):
+        plan = _plan(dg, 1, pc["M"], N, K, pc["G"])
+        assert (plan["BN"], plan["stages"], plan["ks"], plan["pair"]) == ("256", "4", "1", "0"), plan
+        A, sA, B, sB, D, mi = dev_contiguous(pc)
+        dg.dg_fp8_grouped_gemm_contiguous(A, sA, B, sB, D, mi)
+        plan = _plan(dg, 2, max_m, N, K, G)
+        assert (plan["BN"], plan["stages"], plan["ks"], plan["pair"]) == ("256", "4", "1", "0"), plan
+        Am, sAm, Bm, sBm, Dm, m = dev_masked(pm)
+        dg.dg_fp8_grouped_gemm_masked(Am, sAm, Bm, sBm, Dm, m, max_m)
+        st = dg.dg_get_device_status()
+    assert st == 0, dg.dg_status_string(st)
+    got = bits(D)
+    _, ref = oracle_mod.grouped_contiguous(pc["A"], pc["sA"], pc["B"], pc["sB"], pc["m_indices"],
+                                           np.full((pc["M"], N), SENTINEL, np.uint16))
+    pad = pc["m_indices"] < 0
+    assert pad.any()
+    assert np.array_equal(got[pad], ref[pad])
+    assert_close(got[~pad], ref[~pad], "contiguous, four-stage 128x256 tile")
+    got = bits(Dm)
+    _, ref = oracle_mod.grouped_masked(pm["A"], pm["sA"], pm["B"], pm["sB"], pm["masked_m"],
+                                       np.full((G, max_m, N), SENTINEL, np.uint16))
+    valid = np.arange(max_m)[None, :] < mm[:, None]
+    assert np.array_equal(got[~valid], ref[~valid])
+    assert_close(got[valid], ref[valid], "masked, four-stage 128x256 tile")
+
 def test_masked_decode_tile_path(dg, oracle_mod):
     """The planner's own tile for decode-sized masked groups (no width or
     family pinned): 128 columns, three stages of two K blocks, a second
-    producer warp for the B boxes, rows stored directly.  Whole output, with
+    producer warp for the B boxes, rows stored through per-warp buffers.  Whole output, with
     every group's masked rows checked bit for bit; K = 1152 leaves the last
     stage half outside K, and ragged masked_m values cover partial row
     blocks, a group of 128 + 1 rows and an empty group."""
