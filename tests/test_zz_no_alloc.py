@@ -9,8 +9,9 @@ serves them by keeping its K-split partials in a fixed array inside the
 library.  This file checks, through the C ABI, that its results match both
 the CPU oracle and dg_fp8_gemm_nt (within the parity tolerance of the other
 tests) on calls in a row -- each later call finds the previous call's
-partials still in the shared array -- and that its calls make no device
-allocation (the library's own count of cudaMalloc calls does not move).
+partials still in the shared array -- that its calls make no device
+allocation (the library's own count of cudaMalloc calls does not move), and
+that a call captured in a CUDA graph replays correctly.
 
 It sits in a file pytest collects last, so a run that stops at the first
 failure has already run every other test; it also passes alone in a fresh
@@ -72,6 +73,43 @@ def test_noalloc_matches_oracle_and_default_entry_point(dg, oracle_mod, M, N, K)
         assert_close(got, oracle_ref, f"no-alloc call {i + 1} vs oracle, {M}x{N}x{K}")
         assert_close(got, ref, f"no-alloc call {i + 1} vs dg_fp8_gemm_nt, {M}x{N}x{K}")
 
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 2112, 7168), (300, 2112, 1152)])
+def test_noalloc_under_cuda_graph_capture(dg, oracle_mod, M, N, K):
+    """The use the entry point is made for: after one direct call on the
+    device, a call captured in a CUDA graph (global capture mode, in which an
+    allocation or a synchronising call would end the capture with an error)
+    replays to the same bits as the direct call, and, once the captured
+    input tensors are overwritten in place with another problem, to the
+    oracle's result for that problem."""
+    p = gi.dense_problem(M, N, K, seed_a=600 + M, seed_b=700 + N)
+    A, sA, B, sB, D = dev_dense(p)
+    dg.dg_fp8_gemm_nt_noalloc(A, sA, B, sB, D)  # the first call on the device
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    direct = bits(D).copy()
+
+    allocs_before = dg.dg_get_device_allocations()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="global"):
+        dg.dg_fp8_gemm_nt_noalloc(A, sA, B, sB, D)
+    D.view(torch.int16).fill_(0)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    assert np.array_equal(bits(D), direct), "the replayed call differs from the direct call"
+
+    q = gi.dense_problem(M, N, K, seed_a=800 + M, seed_b=900 + N)
+    _, oracle_ref = oracle_mod.gemm_nt(q["A"], q["sA"], q["B"], q["sB"], want_f64=False)
+    for dst, src in zip((A, sA, B, sB), dev_dense(q)[:4]):
+        dst.copy_(src)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert dg.dg_get_device_status() == 0
+    assert dg.dg_get_device_allocations() == allocs_before, "capture or replay allocated"
+    assert_close(bits(D), oracle_ref, f"replayed no-alloc call vs oracle, {M}x{N}x{K}")
+    del graph
 
 def test_noalloc_rejects_problems_beyond_its_scratch(dg):
     # 4096 x 7168 needs 32 x 50 tiles x 73,728 bytes = 118 MB of partials even
